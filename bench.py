@@ -1,0 +1,626 @@
+#!/usr/bin/env python
+"""Benchmark of libssd, the Mamba-2 SSD layer, on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+    torchrun --nproc-per-node N bench.py --gpus N ...     (one process per GPU)
+
+Prints ONE JSON line (rank 0).  The headline is prefill throughput of the 2.7B-shaped
+SSD layer (batch 1, L = 4096, 80 heads x 64 channels, d_state 128, chunk 256, bf16 x/B/C,
+fp32 dt/A/D/state/y): one step = one ssd_prefill of that layer (all four prefill
+kernels).  The batched cached-decode workload (batch 256 x 80 heads, fp32 state
+671 MB, 1024 steps) is reported under "decode" in the same line.
+
+Timing: CUDA events on the launching stream; W untimed warm-up steps; K timed steps
+bracketed by a barrier and a device synchronise on both sides; the max over ranks.  The
+prefill inputs fit in L2, so a 256 MiB buffer is written before every timed prefill step
+(outside that step's events).  The decode state (671 MB) is larger than L2.
+Multi-GPU: every rank runs its own independent sequence (weak scaling), no collective
+on the data path.
+
+`--impl reference` times the fp64 CPU oracle on this machine's cores instead (rank 0
+only), on a bounded sample of the same workload per step.
+"""
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+PREFILL_WORKLOAD = "mamba2_2.7b_prefill"
+DECODE_WORKLOAD = "mamba2_2.7b_decode_b256"
+METRIC = "SSD prefill tokens/s (TFLOP/s) and decode steps/s with HBM GB/s vs peak"
+L2_FLUSH_BYTES = 256 << 20
+FP32_SIMT_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12   # SMs x FP32 lanes x FMA x max clock
+
+
+# ----------------------------------------------------------------------------- helpers
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "bf16_tflops_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                "source": "measured"}
+    except (OSError, KeyError, ValueError):
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                "source": "fallback"}
+
+
+def dist_env():
+    return (int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)),
+            int(os.environ.get("LOCAL_RANK", 0)))
+
+
+def init_dist(world, backend, device=None):
+    import datetime
+    import torch.distributed as dist
+    if world > 1 and not dist.is_initialized():
+        kw = {}
+        if device is not None and backend == "nccl":
+            kw["device_id"] = device
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120), **kw)
+    return dist
+
+
+def barrier(world, device=None):
+    import torch.distributed as dist
+    if world > 1:
+        if device is not None and device.type == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+def max_over_ranks(value: float, world: int, device) -> float:
+    import torch
+    import torch.distributed as dist
+    if world == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def rank_seed(base_seed: int, rank: int) -> int:
+    """Every rank draws its own independent sequence."""
+    return base_seed + 1000 * rank
+
+
+class ClockSampler:
+    """Samples SM clock, power and clock-event reasons through NVML (read-only) while
+    the timed regions run."""
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+    def __init__(self, device_index: int, period_s: float = 0.01):
+        self.samples, self.reasons, self.ok = [], set(), False
+        self.period = period_s
+        self._stop = threading.Event()
+        self._active = threading.Event()
+        self._thread = None
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            self.h = None
+            for i in range(pynvml.nvmlDeviceGetCount()):
+                h = pynvml.nvmlDeviceGetHandleByIndex(i)
+                u = pynvml.nvmlDeviceGetUUID(h)
+                u = u.decode() if isinstance(u, bytes) else u
+                if u.replace("GPU-", "") == uuid.replace("GPU-", ""):
+                    self.h = h
+            if self.h is None:
+                self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # NVML missing: report no clocks rather than guess
+            self.err = repr(e)
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            if self._active.is_set():
+                try:
+                    mhz = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                    try:
+                        r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                    except AttributeError:
+                        r = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+                    self.samples.append(mhz)
+                    for bit, name in self.REASONS.items():
+                        if r & bit and bit != 0x1:
+                            self.reasons.add(name)
+                except Exception:
+                    pass
+            time.sleep(self.period)
+
+    def start(self):
+        if self.ok and self._thread is None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+
+    def active(self, on: bool):
+        (self._active.set if on else self._active.clear)()
+
+    def stop(self):
+        self._stop.set()
+        if self._thread:
+            self._thread.join()
+
+    def summary(self):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "note": "NVML unavailable"}
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                "samples": len(self.samples)}
+
+
+def source_digest(files):
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def profile_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from a committed ncu summary (profiles/<kernel>.<workload>.txt),
+    or None if there is none or the kernel's sources changed since it was taken."""
+    path = os.path.join(ROOT, "profiles", f"{kernel}.{workload}.txt")
+    if not os.path.exists(path):
+        return None
+    kv = {}
+    for line in open(path):
+        if "=" in line and not line.lstrip().startswith("#"):
+            k, v = line.split("=", 1)
+            kv[k.strip()] = v.strip()
+    try:
+        files = kv["sources"].split()
+        if source_digest(files) != kv["sources_sha256"]:
+            return None
+        return float(kv["traffic_bytes_per_launch"])
+    except (KeyError, OSError, ValueError):
+        return None
+
+
+# ------------------------------------------------------------------------ work models
+
+def prefill_work(w, Q=None):
+    """Algorithmic FLOPs and minimum bytes of one prefill of workload w."""
+    Q = Q or w.chunk
+    b, L, H, P, N, G = w.batch, w.seqlen, w.nheads, w.headdim, w.dstate, w.ngroups
+    tok = b * L
+    el = 2 if w.dtype == "bf16" else 4
+    flops_dense = tok * H * (2 * Q * P + 4 * N * P) + tok * G * 2 * Q * N
+    flops_causal = tok * H * ((Q + 1) * P + 4 * N * P) + tok * G * (Q + 1) * N
+    min_bytes = (tok * H * P * el + 2 * tok * G * N * el + tok * H * 4 + 2 * H * 4
+                 + tok * H * P * 4 + b * H * P * N * 4)
+    return flops_dense, flops_causal, min_bytes
+
+
+def kernel_work(name, w, Q):
+    """(bound, algorithmic amount per launch, unit) of one prefill kernel."""
+    b, L, H, P, N, G = w.batch, w.seqlen, w.nheads, w.headdim, w.dstate, w.ngroups
+    tok, nc = b * L, -(-w.seqlen // Q)
+    el = 2 if w.dtype == "bf16" else 4
+    if name.startswith("dA_cumsum"):
+        return "hbm", tok * H * 4 + b * H * nc * Q * 4, "bytes"
+    if name.startswith("state_passing"):
+        return "hbm", 2 * b * nc * H * P * N * 4 + b * H * P * N * 4, "bytes"
+    if name.startswith("chunk_state"):
+        return "flops", tok * H * 2 * N * P, "flops"
+    if name.startswith("chunk_scan"):
+        return "flops", tok * H * (2 * Q * P + 2 * N * P) + tok * G * 2 * Q * N, "flops"
+    return "hbm", 0, "bytes"
+
+
+def roofline_entry(name, w, Q, avg_ms, peaks, traffic):
+    kind, amount, _ = kernel_work(name, w, Q)
+    secs = avg_ms / 1e3
+    if kind == "hbm":
+        achieved = amount / secs / 1e9
+        return {"kernel": name, "bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"], "traffic": traffic,
+                "peak_source": f"{peaks['source']} hbm_gbs"}
+    achieved = amount / secs / 1e12
+    if name.endswith("_simt"):  # fp32 FMA on CUDA cores
+        return {"kernel": name, "bound": "alu", "achieved": achieved, "peak": FP32_SIMT_PEAK_TFLOPS,
+                "unit": "TFLOP/s", "frac": achieved / FP32_SIMT_PEAK_TFLOPS, "traffic": traffic,
+                "peak_source": "148 SMs x 128 FP32 lanes x 2 x 1.965 GHz"}
+    return {"kernel": name, "bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
+            "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"], "traffic": traffic,
+            "peak_source": f"{peaks['source']} bf16_tflops (burst)"}
+
+
+# ------------------------------------------------------------------------ CPU oracle legs
+
+def oracle_prefill_rate(w, seed, min_seconds=10.0, max_seconds=30.0, heads=None):
+    """Oracle tokens/s of the whole layer, timed over repeated runs of a sample (all heads by
+    default).  Returns (tokens_per_s, description, threads, seconds)."""
+    import oracle
+    from selective_state_space_10_b200 import inputs
+    si = inputs.workload_sequence(w, seed=seed)
+    H = w.nheads if heads is None else heads
+    f64 = lambda a: np.ascontiguousarray(a, dtype=np.float64)
+    args = (f64(si.x[:, :, :H]), f64(si.dt[:, :, :H]), f64(si.A[:H]), f64(si.B), f64(si.C), f64(si.D[:H]))
+    threads = oracle.default_threads()
+    reps, spent = 0, 0.0
+    while spent < min_seconds and (reps == 0 or spent * (reps + 1) / reps < max_seconds):
+        t0 = time.perf_counter()
+        oracle.recurrence(*args, nthreads=threads)
+        spent += time.perf_counter() - t0
+        reps += 1
+    tokens = reps * w.batch * w.seqlen * (H / w.nheads)
+    desc = f"{reps} x fp64 recurrence over {H} of {w.nheads} heads x {w.seqlen} tokens (full layer = {w.nheads} heads)"
+    return tokens / spent, desc, threads, spent
+
+
+def oracle_decode_rate(w, seed, min_seconds=10.0, max_seconds=30.0):
+    """Oracle decode steps/s of the whole batch, from repeated steps on all heads."""
+    import oracle
+    from selective_state_space_10_b200 import inputs
+    tok = inputs.decode_token(w, 0, seed=seed)
+    rng = np.random.default_rng(seed)
+    state = rng.standard_normal((w.batch, w.nheads, w.headdim, w.dstate)) * 0.1
+    args = [np.ascontiguousarray(a, dtype=np.float64) for a in (tok.x, tok.dt, tok.A, tok.B, tok.C, tok.D)]
+    threads = oracle.default_threads()
+    reps, spent = 0, 0.0
+    while spent < min_seconds and (reps == 0 or spent * (reps + 1) / reps < max_seconds):
+        t0 = time.perf_counter()
+        _, state = oracle.recurrence(*args, state=state, nthreads=threads)
+        spent += time.perf_counter() - t0
+        reps += 1
+    return reps / spent, f"{reps} fp64 decode steps over all {w.batch}x{w.nheads} heads", threads, spent
+
+
+# ------------------------------------------------------------------------ GPU legs
+
+def upload(si, dev):
+    import torch
+    def inp(name):
+        if si.dtype == "bf16":
+            return torch.from_numpy(si.bits[name].view(np.int16)).view(torch.bfloat16).to(dev)
+        return torch.from_numpy(np.ascontiguousarray(getattr(si, name))).to(dev)
+    f = lambda a: torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(dev)
+    return dict(x=inp("x"), dt=f(si.dt), A=f(si.A), B=inp("B"), C=inp("C"), D=f(si.D))
+
+
+def prefill_leg(args, dev, rank, world, peaks, sampler):
+    import torch
+    from selective_state_space_10_b200 import inputs, ssd
+    w = inputs.BY_NAME[args.workload]
+    si = inputs.workload_sequence(w, seed=rank_seed(w.seed, rank))
+    t = upload(si, dev)
+    dims = ssd.dims_of_prefill(t["x"], t["B"])
+    dtype = ssd.BF16 if w.dtype == "bf16" else ssd.F32
+    names = ssd.prefill_kernel_names(dims, dtype, w.chunk)
+    nk = len(names)
+    ws = torch.empty(ssd.prefill_workspace_size(dims, dtype, w.chunk), dtype=torch.uint8, device=dev)
+    y = torch.empty((w.batch, w.seqlen, w.nheads, w.headdim), dtype=torch.float32, device=dev)
+    fs = torch.empty((w.batch, w.nheads, w.headdim, w.dstate), dtype=torch.float32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    K, W = args.steps, args.warmup
+    mk = lambda: torch.cuda.Event(enable_timing=True)
+    kev = [[mk() for _ in range(nk + 1)] for _ in range(K)]
+    outer = [(mk(), mk()) for _ in range(K)]
+    for evs in kev:          # create the underlying CUDA events before handing them over
+        for e in evs:
+            e.record(stream)
+    for a, b in outer:
+        a.record(stream)
+        b.record(stream)
+    call = lambda events=None: ssd.prefill(**t, chunk=w.chunk, y=y, final_state=fs, workspace=ws,
+                                           stream=stream, events=events)
+    for i in range(W):
+        flush.fill_(i & 0xFF)
+        call()
+    torch.cuda.synchronize(dev)
+    barrier(world, dev)
+    torch.cuda.synchronize(dev)
+    sampler.active(True)
+    for k in range(K):
+        flush.fill_((k + 7) & 0xFF)
+        outer[k][0].record(stream)
+        call(events=kev[k])
+        outer[k][1].record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world, dev)
+    sampler.active(False)
+    step_ms = [a.elapsed_time(b) for a, b in outer]
+    kern_ms = [[kev[k][i].elapsed_time(kev[k][i + 1]) for k in range(K)] for i in range(nk)]
+    total_ms = max_over_ranks(sum(step_ms), world, dev)
+    ms_per_step = total_ms / K
+    tokens = w.batch * w.seqlen
+    value = world * tokens * K / (total_ms / 1e3)
+    fl_dense, fl_causal, min_bytes = prefill_work(w)
+    secs = ms_per_step / 1e3
+    avg = {n: statistics.mean(kern_ms[i]) for i, n in enumerate(names)}
+    tot = sum(avg.values())
+    dom = max(avg, key=avg.get)
+    kernel_srcs = {n: ["selective_state_space_10_b200/csrc/prefill_simt.cu"] for n in names}
+    res = {
+        "value": value, "ms_per_step": ms_per_step, "tokens_per_step_per_gpu": tokens,
+        "tflops": {"dense_tile": fl_dense / secs / 1e12, "causal_only": fl_causal / secs / 1e12,
+                   "frac_of_bf16_peak_dense_tile": fl_dense / secs / 1e12 / peaks["bf16_tflops"],
+                   "peak": peaks["bf16_tflops"], "peak_source": f"{peaks['source']} bf16_tflops (burst)"},
+        "hbm": {"min_bytes": min_bytes, "GB/s": min_bytes / secs / 1e9,
+                "frac": min_bytes / secs / 1e9 / peaks["hbm_gbs"], "peak": peaks["hbm_gbs"]},
+        "kernels": {n: {"avg_ms": avg[n], "share": avg[n] / tot} for n in names},
+        "roofline": roofline_entry(dom, w, w.chunk, avg[dom], peaks, profile_traffic(dom, w.name)),
+        "gpu_launches": K * nk,
+        "config": {"workload": w.name, "batch": w.batch, "seqlen": w.seqlen, "nheads": w.nheads,
+                   "headdim": w.headdim, "dstate": w.dstate, "ngroups": w.ngroups, "chunk": w.chunk,
+                   "input_dtype": w.dtype, "y_dtype": "f32",
+                   "l2": "256 MiB buffer written before every timed step (not timed): inputs fit in L2",
+                   "parallelism": f"{world} GPU(s), one independent sequence per GPU, no collective"},
+    }
+    _ = kernel_srcs
+    # End to end: pinned host inputs -> device, prefill, y and final state -> pinned host.
+    host = {k: v.cpu().pin_memory() for k, v in t.items()}
+    y_h = torch.empty(y.shape, dtype=y.dtype, pin_memory=True)
+    fs_h = torch.empty(fs.shape, dtype=fs.dtype, pin_memory=True)
+    dev_in = {k: torch.empty_like(v) for k, v in t.items()}
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = y.numel() * 4 + fs.numel() * 4
+    ke = max(3, min(K, 20))
+
+    def e2e_step():
+        for k in host:
+            dev_in[k].copy_(host[k], non_blocking=True)
+        ssd.prefill(**dev_in, chunk=w.chunk, y=y, final_state=fs, workspace=ws, stream=stream)
+        y_h.copy_(y, non_blocking=True)
+        fs_h.copy_(fs, non_blocking=True)
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    barrier(world, dev)
+    a, b = mk(), mk()
+    a.record(stream)
+    for _ in range(ke):
+        e2e_step()
+    b.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world, dev)
+    e2e_ms = max_over_ranks(a.elapsed_time(b), world, dev)
+    res["e2e"] = {"value": world * tokens * ke / (e2e_ms / 1e3), "unit": "tokens/s", "steps": ke,
+                  "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                  "path": "pinned host tensors -> device copies -> ssd_prefill -> y, final_state -> pinned host"}
+    return res
+
+
+def decode_leg(args, dev, rank, world, peaks, sampler):
+    import torch
+    from selective_state_space_10_b200 import inputs, ssd
+    w = inputs.BY_NAME[DECODE_WORKLOAD]
+    seed = rank_seed(w.seed, rank)
+    nsteps = args.decode_steps
+    state = torch.from_numpy(inputs.decode_initial_state(w, seed=seed)).to(dev)
+    b, H, P, N, G = w.batch, w.nheads, w.headdim, w.dstate, w.ngroups
+    xs = torch.empty((nsteps, b, H, P), dtype=torch.bfloat16, device=dev)
+    dts = torch.empty((nsteps, b, H), dtype=torch.float32, device=dev)
+    Bs = torch.empty((nsteps, b, G, N), dtype=torch.bfloat16, device=dev)
+    Cs = torch.empty((nsteps, b, G, N), dtype=torch.bfloat16, device=dev)
+    A = D = None
+    for k in range(nsteps):
+        tok = inputs.decode_token(w, k, seed=seed)
+        bf = lambda n: torch.from_numpy(tok.bits[n].view(np.int16)).view(torch.bfloat16)
+        xs[k].copy_(bf("x")[:, 0])
+        dts[k].copy_(torch.from_numpy(tok.dt[:, 0]))
+        Bs[k].copy_(bf("B")[:, 0])
+        Cs[k].copy_(bf("C")[:, 0])
+        if A is None:
+            A = torch.from_numpy(tok.A).to(dev)
+            D = torch.from_numpy(tok.D).to(dev)
+    y = torch.empty((b, H, P), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    step = lambda k: ssd.decode_step(state, xs[k], dts[k], A, Bs[k], Cs[k], D, y=y, stream=stream)
+    for k in range(args.warmup):
+        step(k % nsteps)
+    torch.cuda.synchronize(dev)
+    mk = lambda: torch.cuda.Event(enable_timing=True)
+    # (1) plain launches, back to back
+    barrier(world, dev)
+    torch.cuda.synchronize(dev)
+    sampler.active(True)
+    a, e = mk(), mk()
+    a.record(stream)
+    for k in range(nsteps):
+        step(k)
+    e.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world, dev)
+    sampler.active(False)
+    plain_ms = max_over_ranks(a.elapsed_time(e), world, dev)
+    # (2) the same steps captured once in a CUDA graph and replayed
+    g = torch.cuda.CUDAGraph()
+    cap = torch.cuda.Stream(dev)
+    cap.wait_stream(stream)
+    with torch.cuda.stream(cap):
+        with torch.cuda.graph(g, stream=cap):
+            for k in range(nsteps):
+                ssd.decode_step(state, xs[k], dts[k], A, Bs[k], Cs[k], D, y=y, stream=cap)
+    torch.cuda.synchronize(dev)
+    g.replay()
+    torch.cuda.synchronize(dev)
+    barrier(world, dev)
+    torch.cuda.synchronize(dev)
+    sampler.active(True)
+    a, e = mk(), mk()
+    a.record(stream)
+    g.replay()
+    e.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world, dev)
+    sampler.active(False)
+    graph_ms = max_over_ranks(a.elapsed_time(e), world, dev)
+    del g
+    state_bytes = b * H * P * N * 4
+    step_bytes = 2 * state_bytes + b * H * P * (2 + 4) + b * H * 4 + 2 * b * G * N * 2 + 2 * H * 4
+    best_ms = min(plain_ms, graph_ms) / nsteps
+    gbs = step_bytes / (best_ms / 1e3) / 1e9
+    res = {
+        "workload": w.name, "value": world * nsteps / (min(plain_ms, graph_ms) / 1e3), "unit": "steps/s",
+        "ms_per_step": best_ms, "steps": nsteps, "plain_ms_per_step": plain_ms / nsteps,
+        "graph_ms_per_step": graph_ms / nsteps, "bytes_per_step": step_bytes, "GB/s": gbs,
+        "frac_of_hbm_peak": gbs / peaks["hbm_gbs"],
+        "roofline": {"kernel": "decode_step", "bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"],
+                     "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"],
+                     "traffic": profile_traffic("decode_step", w.name),
+                     "peak_source": f"{peaks['source']} hbm_gbs",
+                     "duration": "per-launch average over back-to-back launches (CUDA graph replay if faster)"},
+        "gpu_launches": nsteps,
+        "config": {"workload": w.name, "batch": b, "nheads": H, "headdim": P, "dstate": N, "ngroups": G,
+                   "input_dtype": "bf16", "state_dtype": "f32", "y_dtype": "f32",
+                   "l2": "state (671 MB) larger than L2; no flush"},
+    }
+    # End to end: per step, the step's inputs from pinned host memory and y back.
+    ke = min(nsteps, 64)
+    hx = xs[:ke].cpu().pin_memory()
+    hdt = dts[:ke].cpu().pin_memory()
+    hB = Bs[:ke].cpu().pin_memory()
+    hC = Cs[:ke].cpu().pin_memory()
+    y_h = torch.empty((ke,) + tuple(y.shape), dtype=y.dtype, pin_memory=True)
+    dx, ddt, dB, dC = (torch.empty_like(xs[0]), torch.empty_like(dts[0]), torch.empty_like(Bs[0]),
+                       torch.empty_like(Cs[0]))
+    torch.cuda.synchronize(dev)
+    barrier(world, dev)
+    a, e = mk(), mk()
+    a.record(stream)
+    for k in range(ke):
+        dx.copy_(hx[k], non_blocking=True)
+        ddt.copy_(hdt[k], non_blocking=True)
+        dB.copy_(hB[k], non_blocking=True)
+        dC.copy_(hC[k], non_blocking=True)
+        ssd.decode_step(state, dx, ddt, A, dB, dC, D, y=y, stream=stream)
+        y_h[k].copy_(y, non_blocking=True)
+    e.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world, dev)
+    e2e_ms = max_over_ranks(a.elapsed_time(e), world, dev)
+    res["e2e"] = {"value": world * ke / (e2e_ms / 1e3), "unit": "steps/s", "steps": ke,
+                  "h2d_bytes_per_step": dx.numel() * 2 + ddt.numel() * 4 + dB.numel() * 2 + dC.numel() * 2,
+                  "d2h_bytes_per_step": y.numel() * 4,
+                  "path": "pinned host x, dt, B, C -> device -> ssd_decode_step -> y -> pinned host"}
+    return res
+
+
+def run_ours(args):
+    import torch
+    rank, world, local = dist_env()
+    if world != args.gpus:
+        if args.gpus > 1 and world == 1:
+            print(json.dumps({"error": f"--gpus {args.gpus} needs torchrun with {args.gpus} processes"}))
+            return 2
+    if not torch.cuda.is_available():
+        print(json.dumps({"error": "no CUDA device: libssd has no CPU path"}))
+        return 2
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    init_dist(world, "nccl", dev)
+    peaks = load_peaks()
+    sampler = ClockSampler(local)
+    sampler.start()
+    try:
+        pre = prefill_leg(args, dev, rank, world, peaks, sampler)
+        dec = None if args.skip_decode else decode_leg(args, dev, rank, world, peaks, sampler)
+    finally:
+        sampler.stop()
+    from selective_state_space_10_b200 import inputs
+    out = {
+        "metric": METRIC, "value": pre["value"], "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": pre["ms_per_step"], "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded; value recipe in inputs.py)",
+        "config": pre["config"], "tflops": pre["tflops"], "hbm": pre["hbm"], "kernels": pre["kernels"],
+        "roofline": pre["roofline"], "gpu_launches": pre["gpu_launches"] + (dec["gpu_launches"] if dec else 0),
+        "gpu_launches_prefill_timed_region": pre["gpu_launches"], "e2e": pre["e2e"],
+        "peaks": peaks, "clocks": sampler.summary(), "impl": "ours",
+    }
+    if dec:
+        out["decode"] = dec
+    if rank == 0 and world == 1 and not args.skip_cpu_baseline:
+        w = inputs.BY_NAME[args.workload]
+        rate, desc, threads, secs = oracle_prefill_rate(w, w.seed)
+        out["cpu_baseline"] = {"value": rate, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                               "sample": desc, "seconds": secs}
+        if dec:
+            wd = inputs.BY_NAME[DECODE_WORKLOAD]
+            drate, ddesc, dthreads, dsecs = oracle_decode_rate(wd, wd.seed)
+            out["decode"]["cpu_baseline"] = {"value": drate, "unit": "steps/s", "cores": dthreads,
+                                             "kind": "oracle", "sample": ddesc, "seconds": dsecs}
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+def run_reference(args):
+    """The fp64 CPU oracle as the reference arm: rank 0 only, K timed steps of a bounded
+    sample (16 of 80 heads, all 4096 tokens) of the prefill workload per step."""
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    import oracle
+    from selective_state_space_10_b200 import inputs
+    w = inputs.BY_NAME[args.workload]
+    si = inputs.workload_sequence(w)
+    Hs = min(16, w.nheads)
+    f64 = lambda a: np.ascontiguousarray(a, dtype=np.float64)
+    a = (f64(si.x[:, :, :Hs]), f64(si.dt[:, :, :Hs]), f64(si.A[:Hs]), f64(si.B), f64(si.C), f64(si.D[:Hs]))
+    threads = oracle.default_threads()
+    for _ in range(args.warmup):
+        oracle.recurrence(*a, nthreads=threads)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.recurrence(*a, nthreads=threads)
+    secs = time.perf_counter() - t0
+    tokens = args.steps * w.batch * w.seqlen * Hs / w.nheads
+    value = tokens / secs
+    sample = f"per step: fp64 recurrence over {Hs} of {w.nheads} heads x {w.seqlen} tokens; value scaled to the full layer"
+    print(json.dumps({
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": secs / args.steps * 1e3 * w.nheads / Hs, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
+        "config": {"workload": w.name, "batch": w.batch, "seqlen": w.seqlen, "nheads": w.nheads,
+                   "headdim": w.headdim, "dstate": w.dstate, "ngroups": w.ngroups, "chunk": w.chunk},
+        "impl": "reference",
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=PREFILL_WORKLOAD)
+    ap.add_argument("--decode-steps", type=int, default=1024)
+    ap.add_argument("--skip-decode", action="store_true")
+    ap.add_argument("--skip-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    return run_reference(args) if args.impl == "reference" else run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

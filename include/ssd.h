@@ -1,0 +1,172 @@
+/*
+ * ssd.h -- C ABI of libssd, the Mamba-2 state space duality (SSD) layer for NVIDIA B200.
+ *
+ * The layer (per batch row and head h, group g = h / (nheads / ngroups)):
+ *
+ *     a_t      = exp(dt_t * A_h)
+ *     h_t[p,n] = a_t * h_{t-1}[p,n] + dt_t * x_t[p] * B_t[g,n]
+ *     y_t[p]   = sum_n C_t[g,n] * h_t[p,n] + D_h * x_t[p]
+ *
+ * Sources: "Engineering Hybrid State-Space Models" section 2 (the diagonal recurrence
+ * h_t = Abar_t h_{t-1} + Bbar_t x_t, y_t = C_t h_t with Abar_t = exp(dt_t A), and its
+ * chunked semiseparable form Y = (M o C B^T) X); "Compiler-First State Space Duality and
+ * Portable O(1) Autoregressive Caching for Inference" abstract (scalar per-head dynamics,
+ * fixed-size chunking, a prefill that hands an O(1) cache to single-token decode);
+ * "Mamba and Selective State Space Models" section 2 (the D x feedthrough).  The input
+ * term is the Euler form dt_t * B_t (the first page's code section uses delta * x), not
+ * the full zero-order-hold Bbar.
+ *
+ * Layouts (row-major, contiguous, no strides):
+ *     x      [batch, seqlen, nheads, headdim]      dtype of the call (fp32 or bf16)
+ *     dt     [batch, seqlen, nheads]               fp32, > 0 (not checked: device data)
+ *     A      [nheads]                              fp32 (normally < 0)
+ *     B, C   [batch, seqlen, ngroups, dstate]      dtype of the call
+ *     D      [nheads]                              fp32
+ *     y      [batch, seqlen, nheads, headdim]      fp32 (always, see below)
+ *     state  [batch, nheads, headdim, dstate]      fp32
+ * Decode drops the seqlen axis (x [batch, nheads, headdim], dt [batch, nheads], B and C
+ * [batch, ngroups, dstate], y [batch, nheads, headdim]).
+ *
+ * y is written in fp32 for every input dtype: the layer's output is dominated by the
+ * D x term, whose largest elements are many times its RMS, and rounding those to bf16
+ * would by itself exceed a max-error bound of 2e-2 RMS.
+ *
+ * Conventions of every call:
+ *   - All array pointers are DEVICE pointers on the current CUDA device, owned by the
+ *     caller.  libssd never allocates, frees or keeps device memory, and keeps no state
+ *     between calls.  A pointer may be NULL only if its array has zero elements.
+ *   - x, B, C, y, state, final_state and workspace must be 16-byte aligned; dt, A and D
+ *     4-byte aligned.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy default
+ *     stream): they validate on the host, enqueue kernels and return.  On a validation
+ *     error nothing is enqueued.  A launch failure is reported as SSD_ERR_CUDA.  No call
+ *     aborts, prints or synchronises.
+ *   - Inputs and outputs must not overlap, except as stated for ssd_decode_step.
+ */
+#ifndef LIBSSD_SSD_H_
+#define LIBSSD_SSD_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SSD_API __attribute__((visibility("default")))
+#else
+#define SSD_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t, declared without the CUDA headers. */
+typedef struct CUstream_st *ssd_stream_t;
+
+typedef enum {
+  SSD_OK = 0,
+  SSD_ERR_INVALID_ARG = 1, /* NULL pointer, misalignment, bad sizes, nheads % ngroups != 0 */
+  SSD_ERR_UNSUPPORTED = 2, /* valid but outside the compiled shape set (see below)        */
+  SSD_ERR_WORKSPACE = 3,   /* workspace NULL or smaller than ssd_prefill_workspace_size()  */
+  SSD_ERR_CUDA = 4,        /* a CUDA runtime call or kernel launch failed                  */
+  SSD_ERR_TIMEOUT = 5      /* reserved for bounded device-side waits; not returned today    */
+} ssd_status;
+
+typedef enum {
+  SSD_F32 = 0, /* x, B, C in fp32; fp32 arithmetic throughout (no tensor cores)          */
+  SSD_BF16 = 1 /* x, B, C in bf16; bf16 tensor-core products with fp32 accumulation      */
+} ssd_dtype;
+
+typedef struct {
+  int64_t batch;   /* >= 0                                     */
+  int64_t seqlen;  /* >= 0 (ignored by ssd_decode_step)        */
+  int64_t nheads;  /* >= 1, multiple of ngroups                */
+  int64_t headdim; /* P: 1 .. 256                              */
+  int64_t dstate;  /* N: one of 16, 32, 64, 128, 256           */
+  int64_t ngroups; /* >= 1                                     */
+} ssd_dims;
+
+/* Human-readable name of a status code (static storage; never NULL). */
+SSD_API const char *ssd_status_string(ssd_status status);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+SSD_API int ssd_version(void);
+
+/*
+ * Bytes of device workspace ssd_prefill needs for these arguments (0 if the arguments
+ * are invalid or need none).  Depends only on the arguments.
+ */
+SSD_API size_t ssd_prefill_workspace_size(const ssd_dims *dims, ssd_dtype dtype, int chunk);
+
+/*
+ * Number of kernels one ssd_prefill call with these arguments enqueues (-1 if the
+ * arguments are invalid).  For launch accounting only.
+ */
+SSD_API int ssd_prefill_kernel_launches(const ssd_dims *dims, ssd_dtype dtype, int chunk);
+
+/*
+ * Chunked prefill from a zero initial state.
+ *
+ * Computes y for every token of every sequence and writes the state after the last
+ * token, h_{seqlen-1}, to final_state (all zeros when seqlen == 0).  `chunk` (Q) is the
+ * chunk length of the chunked form: a power of two in [1, 256]; the result does not
+ * depend on it beyond rounding ("Engineering Hybrid State-Space Models" section 2 uses
+ * Q = 64).  seqlen need not be a multiple of chunk: the last chunk may be partial.
+ *
+ * Within each chunk the kernels compute the in-chunk cumulative log-decay, the chunk's
+ * state contribution, carry the state across chunks, then form each token's output from
+ * the masked decay-weighted C B^T product plus the carried-in state.
+ *
+ * workspace: device scratch of at least ssd_prefill_workspace_size() bytes, 16-byte
+ * aligned, owned by the caller, contents on entry ignored and on return unspecified.
+ * Calls that share a workspace must be ordered (same stream or synchronised).
+ *
+ * Errors: SSD_ERR_INVALID_ARG for NULL dims, NULL or misaligned non-empty arrays,
+ * negative sizes, headdim outside 1..256, nheads % ngroups != 0, chunk not a power of
+ * two in [1, 256]; SSD_ERR_UNSUPPORTED for a dstate outside {16,32,64,128,256};
+ * SSD_ERR_WORKSPACE for a missing or short workspace; SSD_ERR_CUDA if a launch fails.
+ */
+SSD_API ssd_status ssd_prefill(const ssd_dims *dims, ssd_dtype dtype, const void *x, const float *dt,
+                       const float *A, const void *B, const void *C, const float *D,
+                       int chunk, float *y, float *final_state, void *workspace,
+                       size_t workspace_bytes, ssd_stream_t stream);
+
+/*
+ * ssd_prefill, with per-kernel timing for profiling harnesses.  `events` holds
+ * num_events caller-created cudaEvent_t handles (cudaEventDefault flags, i.e. timing
+ * enabled), num_events >= ssd_prefill_kernel_launches() + 1.  events[i] is recorded on
+ * `stream` just before kernel i is enqueued and events[k] after the last of the k
+ * kernels, so cudaEventElapsedTime(events[i], events[i+1]) is kernel i's duration.
+ * Nothing is allocated and nothing synchronises.  Same computation, results and errors
+ * as ssd_prefill, plus SSD_ERR_INVALID_ARG if events is NULL or too short.
+ */
+SSD_API ssd_status ssd_prefill_timed(const ssd_dims *dims, ssd_dtype dtype, const void *x, const float *dt,
+                                     const float *A, const void *B, const void *C, const float *D, int chunk,
+                                     float *y, float *final_state, void *workspace, size_t workspace_bytes,
+                                     ssd_stream_t stream, void *const *events, int num_events);
+
+/*
+ * Name of kernel i (0-based) of an ssd_prefill call with these arguments, in launch
+ * order (static storage), or NULL if i is out of range or the arguments are invalid.
+ */
+SSD_API const char *ssd_prefill_kernel_name(const ssd_dims *dims, ssd_dtype dtype, int chunk, int i);
+
+/*
+ * One cached decode step (O(1) in the sequence length: "Compiler-First State Space
+ * Duality ..." abstract; the recurrent mode of "Mamba and Selective State Space Models"
+ * section 3).  Reads state = h_{t-1}, overwrites it in place with h_t, writes y_t.
+ * dims->seqlen is ignored.  Each head's state is read once and written once.
+ *
+ * The state continues a prefill: pass ssd_prefill's final_state to continue that
+ * sequence; any fp32 state (a saved cache) may be passed.
+ *
+ * Errors: as ssd_prefill, without the chunk and workspace checks.
+ */
+SSD_API ssd_status ssd_decode_step(const ssd_dims *dims, ssd_dtype dtype, float *state, const void *x,
+                           const float *dt, const float *A, const void *B, const void *C,
+                           const float *D, float *y, ssd_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LIBSSD_SSD_H_ */

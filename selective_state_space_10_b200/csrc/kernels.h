@@ -1,0 +1,31 @@
+// kernels.h -- host-side launchers of the libssd kernels (internal to the library).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+
+#include "common.cuh"
+
+namespace ssd {
+
+// prefill_simt.cu
+cudaError_t launch_dA_cumsum(const float *dt, const float *A, float *cum, const Dims &d, int Q, int nc,
+                             cudaStream_t st);
+template <typename T>
+cudaError_t launch_chunk_state_simt(const T *x, const float *dt, const T *B, const float *cum, float *states,
+                                    const Dims &d, int Q, int nc, cudaStream_t st);
+cudaError_t launch_state_passing(float *states, const float *cum, float *final_state, const Dims &d, int Q,
+                                 int nc, cudaStream_t st);
+template <typename T>
+cudaError_t launch_chunk_scan_simt(const T *x, const float *dt, const T *B, const T *C, const float *D,
+                                   const float *cum, const float *hprev, float *y, const Dims &d, int Q, int nc,
+                                   cudaStream_t st);
+size_t chunk_scan_simt_smem_bytes(int N);
+
+// decode.cu
+template <typename T>
+cudaError_t launch_decode_step(float *state, const T *x, const float *dt, const float *A, const T *B,
+                               const T *C, const float *D, float *y, const Dims &d, cudaStream_t st);
+
+}  // namespace ssd

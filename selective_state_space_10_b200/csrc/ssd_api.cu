@@ -1,0 +1,225 @@
+// ssd_api.cu -- the C ABI of libssd (include/ssd.h): host-side validation, workspace
+// layout and kernel dispatch.  Every entry point validates all arguments before it
+// enqueues anything; validation makes no CUDA call, so it behaves the same on a host
+// without a GPU.
+#include <stdint.h>
+#include <string.h>
+
+#include "../../include/ssd.h"
+#include "kernels.h"
+
+namespace {
+
+using ssd::Dims;
+
+constexpr int kVersion = 100;  // 0.1.0
+constexpr size_t kAlign = 256;
+
+size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
+
+bool aligned(const void *p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+bool is_pow2(int v) { return v > 0 && (v & (v - 1)) == 0; }
+
+bool supported_dstate(int64_t n) { return n == 16 || n == 32 || n == 64 || n == 128 || n == 256; }
+
+// Shape checks shared by both calls.  Returns SSD_OK and fills `d` on success.
+ssd_status check_dims(const ssd_dims *dims, ssd_dtype dtype, bool prefill, Dims *d) {
+  if (!dims) return SSD_ERR_INVALID_ARG;
+  if (dtype != SSD_F32 && dtype != SSD_BF16) return SSD_ERR_INVALID_ARG;
+  const int64_t lim = (int64_t)1 << 30;
+  if (dims->batch < 0 || dims->batch > lim) return SSD_ERR_INVALID_ARG;
+  if (prefill && (dims->seqlen < 0 || dims->seqlen > lim)) return SSD_ERR_INVALID_ARG;
+  if (dims->nheads < 1 || dims->nheads > 65535) return SSD_ERR_INVALID_ARG;
+  if (dims->ngroups < 1 || dims->nheads % dims->ngroups != 0) return SSD_ERR_INVALID_ARG;
+  if (dims->headdim < 1 || dims->headdim > 256) return SSD_ERR_INVALID_ARG;
+  if (dims->dstate < 1) return SSD_ERR_INVALID_ARG;
+  if (!supported_dstate(dims->dstate)) return SSD_ERR_UNSUPPORTED;
+  // Element counts must stay far from 64-bit overflow and grid limits.
+  const int64_t L = prefill ? dims->seqlen : 1;
+  const double xs = (double)dims->batch * (double)L * (double)dims->nheads * (double)dims->headdim;
+  const double ss = (double)dims->batch * (double)dims->nheads * (double)dims->headdim * (double)dims->dstate;
+  if (xs > 4e12 || ss > 4e12) return SSD_ERR_INVALID_ARG;
+  if ((double)dims->batch * (double)dims->nheads > 2147483647.0) return SSD_ERR_INVALID_ARG;
+  d->b = (int)dims->batch;
+  d->L = prefill ? (int)dims->seqlen : 1;
+  d->H = (int)dims->nheads;
+  d->P = (int)dims->headdim;
+  d->N = (int)dims->dstate;
+  d->G = (int)dims->ngroups;
+  d->hpg = d->H / d->G;
+  return SSD_OK;
+}
+
+// Every non-empty array must be non-NULL and aligned.
+bool check_ptr(const void *p, int64_t elems, size_t align) {
+  if (elems == 0) return true;
+  return p != nullptr && aligned(p, align);
+}
+
+struct PrefillPlan {
+  int nc = 0;            // chunks per sequence
+  size_t cum_off = 0;    // float [b][H][nc][Q]
+  size_t states_off = 0; // float [b][nc][H][P][N]
+  size_t bytes = 0;
+  int launches = 0;
+};
+
+PrefillPlan plan_prefill(const Dims &d, int Q) {
+  PrefillPlan pl;
+  pl.nc = (int)(((int64_t)d.L + Q - 1) / Q);
+  if (d.b == 0 || d.L == 0) return pl;
+  pl.cum_off = 0;
+  pl.states_off = align_up((size_t)d.b * d.H * pl.nc * Q * sizeof(float));
+  pl.bytes = pl.states_off + align_up((size_t)d.b * pl.nc * d.H * (size_t)d.P * d.N * sizeof(float));
+  pl.launches = 4;
+  return pl;
+}
+
+ssd_status cuda_status(cudaError_t e) { return e == cudaSuccess ? SSD_OK : SSD_ERR_CUDA; }
+
+// Records events[i] before kernel i (and events[k] after the last) when events != NULL.
+struct Marker {
+  cudaEvent_t const *ev;
+  cudaStream_t st;
+  int i = 0;
+  cudaError_t mark() { return ev ? cudaEventRecord(ev[i++], st) : cudaSuccess; }
+};
+
+template <typename T>
+ssd_status run_prefill(const Dims &d, int Q, const PrefillPlan &pl, const T *x, const float *dt,
+                       const float *A, const T *B, const T *C, const float *D, float *y, float *final_state,
+                       char *ws, cudaStream_t st, cudaEvent_t const *ev) {
+  float *cum = reinterpret_cast<float *>(ws + pl.cum_off);
+  float *states = reinterpret_cast<float *>(ws + pl.states_off);
+  Marker m{ev, st};
+  cudaError_t e = m.mark();
+  if (e == cudaSuccess) e = ssd::launch_dA_cumsum(dt, A, cum, d, Q, pl.nc, st);
+  if (e == cudaSuccess) e = m.mark();
+  if (e == cudaSuccess) e = ssd::launch_chunk_state_simt<T>(x, dt, B, cum, states, d, Q, pl.nc, st);
+  if (e == cudaSuccess) e = m.mark();
+  if (e == cudaSuccess) e = ssd::launch_state_passing(states, cum, final_state, d, Q, pl.nc, st);
+  if (e == cudaSuccess) e = m.mark();
+  if (e == cudaSuccess) e = ssd::launch_chunk_scan_simt<T>(x, dt, B, C, D, cum, states, y, d, Q, pl.nc, st);
+  if (e == cudaSuccess) e = m.mark();
+  return cuda_status(e);
+}
+
+const char *const kSimtKernelNames[] = {"dA_cumsum", "chunk_state_simt", "state_passing", "chunk_scan_simt"};
+
+}  // namespace
+
+extern "C" {
+
+const char *ssd_status_string(ssd_status s) {
+  switch (s) {
+    case SSD_OK: return "SSD_OK";
+    case SSD_ERR_INVALID_ARG: return "SSD_ERR_INVALID_ARG: invalid argument";
+    case SSD_ERR_UNSUPPORTED: return "SSD_ERR_UNSUPPORTED: shape outside the supported set";
+    case SSD_ERR_WORKSPACE: return "SSD_ERR_WORKSPACE: workspace missing or too small";
+    case SSD_ERR_CUDA: return "SSD_ERR_CUDA: CUDA launch or runtime error";
+    case SSD_ERR_TIMEOUT: return "SSD_ERR_TIMEOUT: bounded device wait expired";
+  }
+  return "unknown ssd_status";
+}
+
+int ssd_version(void) { return kVersion; }
+
+size_t ssd_prefill_workspace_size(const ssd_dims *dims, ssd_dtype dtype, int chunk) {
+  Dims d;
+  if (check_dims(dims, dtype, true, &d) != SSD_OK) return 0;
+  if (!is_pow2(chunk) || chunk > 256) return 0;
+  return plan_prefill(d, chunk).bytes;
+}
+
+int ssd_prefill_kernel_launches(const ssd_dims *dims, ssd_dtype dtype, int chunk) {
+  Dims d;
+  if (check_dims(dims, dtype, true, &d) != SSD_OK) return -1;
+  if (!is_pow2(chunk) || chunk > 256) return -1;
+  return plan_prefill(d, chunk).launches;
+}
+
+static ssd_status prefill_impl(const ssd_dims *dims, ssd_dtype dtype, const void *x, const float *dt,
+                               const float *A, const void *B, const void *C, const float *D, int chunk, float *y,
+                               float *final_state, void *workspace, size_t workspace_bytes, ssd_stream_t stream,
+                               void *const *events, int num_events, bool timed) {
+  Dims d;
+  ssd_status s = check_dims(dims, dtype, true, &d);
+  if (s != SSD_OK) return s;
+  if (!is_pow2(chunk) || chunk > 256) return SSD_ERR_INVALID_ARG;
+  const int64_t ntok = (int64_t)d.b * d.L;
+  const int64_t nx = ntok * d.H * d.P, nbc = ntok * d.G * d.N, nst = (int64_t)d.b * d.H * d.P * d.N;
+  if (!check_ptr(x, nx, 16) || !check_ptr(B, nbc, 16) || !check_ptr(C, nbc, 16) || !check_ptr(y, nx, 16) ||
+      !check_ptr(dt, ntok * d.H, 4) || !check_ptr(final_state, nst, 16))
+    return SSD_ERR_INVALID_ARG;
+  const bool any_heads = d.b > 0 && d.L > 0;
+  if (!check_ptr(A, any_heads ? d.H : 0, 4) || !check_ptr(D, any_heads ? d.H : 0, 4)) return SSD_ERR_INVALID_ARG;
+  const PrefillPlan pl = plan_prefill(d, chunk);
+  if (timed) {
+    if (events == nullptr || num_events < pl.launches + 1) return SSD_ERR_INVALID_ARG;
+    for (int i = 0; i < pl.launches + 1; ++i)
+      if (events[i] == nullptr) return SSD_ERR_INVALID_ARG;
+  }
+  if (pl.bytes > 0 && (workspace == nullptr || !aligned(workspace, 16) || workspace_bytes < pl.bytes))
+    return SSD_ERR_WORKSPACE;
+
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (d.b == 0) return SSD_OK;
+  if (d.L == 0) return cuda_status(cudaMemsetAsync(final_state, 0, (size_t)nst * sizeof(float), st));
+  char *ws = static_cast<char *>(workspace);
+  cudaEvent_t const *ev = timed ? reinterpret_cast<cudaEvent_t const *>(events) : nullptr;
+  if (dtype == SSD_F32)
+    return run_prefill<float>(d, chunk, pl, static_cast<const float *>(x), dt, A, static_cast<const float *>(B),
+                              static_cast<const float *>(C), D, y, final_state, ws, st, ev);
+  return run_prefill<__nv_bfloat16>(d, chunk, pl, static_cast<const __nv_bfloat16 *>(x), dt, A,
+                                    static_cast<const __nv_bfloat16 *>(B), static_cast<const __nv_bfloat16 *>(C), D,
+                                    y, final_state, ws, st, ev);
+}
+
+ssd_status ssd_prefill(const ssd_dims *dims, ssd_dtype dtype, const void *x, const float *dt, const float *A,
+                       const void *B, const void *C, const float *D, int chunk, float *y, float *final_state,
+                       void *workspace, size_t workspace_bytes, ssd_stream_t stream) {
+  return prefill_impl(dims, dtype, x, dt, A, B, C, D, chunk, y, final_state, workspace, workspace_bytes, stream,
+                      nullptr, 0, false);
+}
+
+ssd_status ssd_prefill_timed(const ssd_dims *dims, ssd_dtype dtype, const void *x, const float *dt, const float *A,
+                             const void *B, const void *C, const float *D, int chunk, float *y, float *final_state,
+                             void *workspace, size_t workspace_bytes, ssd_stream_t stream, void *const *events,
+                             int num_events) {
+  return prefill_impl(dims, dtype, x, dt, A, B, C, D, chunk, y, final_state, workspace, workspace_bytes, stream,
+                      events, num_events, true);
+}
+
+const char *ssd_prefill_kernel_name(const ssd_dims *dims, ssd_dtype dtype, int chunk, int i) {
+  Dims d;
+  if (check_dims(dims, dtype, true, &d) != SSD_OK || !is_pow2(chunk) || chunk > 256) return nullptr;
+  const PrefillPlan pl = plan_prefill(d, chunk);
+  if (i < 0 || i >= pl.launches) return nullptr;
+  return kSimtKernelNames[i];
+}
+
+ssd_status ssd_decode_step(const ssd_dims *dims, ssd_dtype dtype, float *state, const void *x, const float *dt,
+                           const float *A, const void *B, const void *C, const float *D, float *y,
+                           ssd_stream_t stream) {
+  Dims d;
+  ssd_status s = check_dims(dims, dtype, false, &d);
+  if (s != SSD_OK) return s;
+  const int64_t nx = (int64_t)d.b * d.H * d.P, nbc = (int64_t)d.b * d.G * d.N;
+  const int64_t nst = (int64_t)d.b * d.H * d.P * d.N;
+  const int64_t nh = d.b > 0 ? d.H : 0;
+  if (!check_ptr(state, nst, 16) || !check_ptr(x, nx, 16) || !check_ptr(B, nbc, 16) || !check_ptr(C, nbc, 16) ||
+      !check_ptr(y, nx, 16) || !check_ptr(dt, (int64_t)d.b * d.H, 4) || !check_ptr(A, nh, 4) || !check_ptr(D, nh, 4))
+    return SSD_ERR_INVALID_ARG;
+  if (d.b == 0) return SSD_OK;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (dtype == SSD_F32)
+    return cuda_status(ssd::launch_decode_step<float>(state, static_cast<const float *>(x), dt, A,
+                                                      static_cast<const float *>(B), static_cast<const float *>(C),
+                                                      D, y, d, st));
+  return cuda_status(ssd::launch_decode_step<__nv_bfloat16>(
+      state, static_cast<const __nv_bfloat16 *>(x), dt, A, static_cast<const __nv_bfloat16 *>(B),
+      static_cast<const __nv_bfloat16 *>(C), D, y, d, st));
+}
+
+}  // extern "C"

@@ -1,0 +1,211 @@
+"""Python binding of libssd (include/ssd.h): argument marshalling only.
+
+Every step of the layer runs in the library's CUDA kernels; this module checks tensor
+devices, dtypes and shapes, allocates outputs with torch when the caller passes none,
+and forwards raw device pointers and the current CUDA stream through ctypes.  Importing
+it loads libssd.so and raises if the library has not been built: there is no fallback.
+"""
+import ctypes
+import os
+from typing import Optional, Tuple
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libssd.so")
+
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_TIMEOUT = range(6)
+F32, BF16 = 0, 1
+_DTYPES = {torch.float32: F32, torch.bfloat16: BF16}
+
+
+class SSDError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)}")
+
+
+class Dims(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int64), ("seqlen", ctypes.c_int64), ("nheads", ctypes.c_int64),
+                ("headdim", ctypes.c_int64), ("dstate", ctypes.c_int64), ("ngroups", ctypes.c_int64)]
+
+
+# Every symbol include/ssd.h declares.
+EXPORTS = ("ssd_status_string", "ssd_version", "ssd_prefill_workspace_size",
+           "ssd_prefill_kernel_launches", "ssd_prefill", "ssd_prefill_timed",
+           "ssd_prefill_kernel_name", "ssd_decode_step")
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"libssd.so is not built ({LIB_PATH}); run "
+                          "`python -m selective_state_space_10_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, fp, i64, ci, sz = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
+    dp = ctypes.POINTER(Dims)
+    lib.ssd_status_string.argtypes = [ci]
+    lib.ssd_status_string.restype = ctypes.c_char_p
+    lib.ssd_version.argtypes = []
+    lib.ssd_version.restype = ci
+    lib.ssd_prefill_workspace_size.argtypes = [dp, ci, ci]
+    lib.ssd_prefill_workspace_size.restype = sz
+    lib.ssd_prefill_kernel_launches.argtypes = [dp, ci, ci]
+    lib.ssd_prefill_kernel_launches.restype = ci
+    lib.ssd_prefill.argtypes = [dp, ci, vp, fp, fp, vp, vp, fp, ci, fp, fp, vp, sz, vp]
+    lib.ssd_prefill.restype = ci
+    lib.ssd_prefill_timed.argtypes = [dp, ci, vp, fp, fp, vp, vp, fp, ci, fp, fp, vp, sz, vp,
+                                      ctypes.POINTER(ctypes.c_void_p), ci]
+    lib.ssd_prefill_timed.restype = ci
+    lib.ssd_prefill_kernel_name.argtypes = [dp, ci, ci, ci]
+    lib.ssd_prefill_kernel_name.restype = ctypes.c_char_p
+    lib.ssd_decode_step.argtypes = [dp, ci, fp, vp, fp, fp, vp, vp, fp, fp, vp]
+    lib.ssd_decode_step.restype = ci
+    return lib
+
+
+lib = _load()
+
+
+def status_string(status: int) -> str:
+    return lib.ssd_status_string(int(status)).decode()
+
+
+def version() -> int:
+    return lib.ssd_version()
+
+
+def _dims(batch, seqlen, nheads, headdim, dstate, ngroups) -> Dims:
+    return Dims(int(batch), int(seqlen), int(nheads), int(headdim), int(dstate), int(ngroups))
+
+
+def dims_of_prefill(x: torch.Tensor, B: torch.Tensor) -> Dims:
+    b, L, H, P = x.shape
+    return _dims(b, L, H, P, B.shape[3], B.shape[2])
+
+
+def prefill_workspace_size(dims: Dims, dtype: int, chunk: int) -> int:
+    return lib.ssd_prefill_workspace_size(ctypes.byref(dims), int(dtype), int(chunk))
+
+
+def prefill_kernel_launches(dims: Dims, dtype: int, chunk: int) -> int:
+    return lib.ssd_prefill_kernel_launches(ctypes.byref(dims), int(dtype), int(chunk))
+
+
+def prefill_kernel_names(dims: Dims, dtype: int, chunk: int):
+    n = prefill_kernel_launches(dims, dtype, chunk)
+    return [lib.ssd_prefill_kernel_name(ctypes.byref(dims), int(dtype), int(chunk), i).decode()
+            for i in range(max(n, 0))]
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _check(t: torch.Tensor, name: str, shape, dtype, device):
+    if t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} has dtype {t.dtype}, expected {dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def prefill(x, dt, A, B, C, D, chunk: int = 256, y=None, final_state=None, workspace=None,
+            stream=None, events=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Chunked prefill from a zero state.  Returns (y fp32 [b,L,H,P], final_state fp32
+    [b,H,P,N]).  x, B, C are fp32 or bf16 (the same dtype); dt, A, D are fp32.
+
+    `events`: optional list of torch.cuda.Event(enable_timing=True), at least
+    prefill_kernel_launches() + 1 of them, already recorded once (so their handles
+    exist); the call then goes through ssd_prefill_timed, which records events[i] before
+    kernel i and events[-1] after the last kernel."""
+    if x.dim() != 4 or B.dim() != 4:
+        raise ValueError("x must be [b,L,H,P] and B, C [b,L,G,N]")
+    if x.dtype not in _DTYPES:
+        raise ValueError(f"unsupported input dtype {x.dtype}")
+    dev = x.device
+    if dev.type != "cuda":
+        raise ValueError("libssd runs on CUDA tensors only")
+    b, L, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    _check(x, "x", (b, L, H, P), x.dtype, dev)
+    _check(dt, "dt", (b, L, H), torch.float32, dev)
+    _check(A, "A", (H,), torch.float32, dev)
+    _check(B, "B", (b, L, G, N), x.dtype, dev)
+    _check(C, "C", (b, L, G, N), x.dtype, dev)
+    _check(D, "D", (H,), torch.float32, dev)
+    if y is None:
+        y = torch.empty((b, L, H, P), dtype=torch.float32, device=dev)
+    if final_state is None:
+        final_state = torch.empty((b, H, P, N), dtype=torch.float32, device=dev)
+    _check(y, "y", (b, L, H, P), torch.float32, dev)
+    _check(final_state, "final_state", (b, H, P, N), torch.float32, dev)
+    dims = dims_of_prefill(x, B)
+    dtype = _DTYPES[x.dtype]
+    need = prefill_workspace_size(dims, dtype, chunk)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    args = (ctypes.byref(dims), dtype, _ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
+            int(chunk), _ptr(y), _ptr(final_state), _ptr(workspace), ws_bytes, _stream(stream))
+    if events is None:
+        st = lib.ssd_prefill(*args)
+    else:
+        handles = (ctypes.c_void_p * len(events))(*[ev.cuda_event for ev in events])
+        st = lib.ssd_prefill_timed(*args, handles, len(events))
+    if st != OK:
+        raise SSDError(st, "ssd_prefill")
+    return y, final_state
+
+
+def decode_step(state, x, dt, A, B, C, D, y=None, stream=None) -> torch.Tensor:
+    """One cached decode step: updates `state` [b,H,P,N] fp32 in place, returns y fp32
+    [b,H,P].  x [b,H,P] and B, C [b,G,N] are fp32 or bf16; dt [b,H], A, D [H] fp32."""
+    if x.dim() != 3 or B.dim() != 3 or state.dim() != 4:
+        raise ValueError("state must be [b,H,P,N], x [b,H,P], B and C [b,G,N]")
+    if x.dtype not in _DTYPES:
+        raise ValueError(f"unsupported input dtype {x.dtype}")
+    dev = x.device
+    if dev.type != "cuda":
+        raise ValueError("libssd runs on CUDA tensors only")
+    b, H, P = x.shape
+    G, N = B.shape[1], B.shape[2]
+    _check(state, "state", (b, H, P, N), torch.float32, dev)
+    _check(dt, "dt", (b, H), torch.float32, dev)
+    _check(A, "A", (H,), torch.float32, dev)
+    _check(B, "B", (b, G, N), x.dtype, dev)
+    _check(C, "C", (b, G, N), x.dtype, dev)
+    _check(D, "D", (H,), torch.float32, dev)
+    if y is None:
+        y = torch.empty((b, H, P), dtype=torch.float32, device=dev)
+    _check(y, "y", (b, H, P), torch.float32, dev)
+    dims = _dims(b, 1, H, P, N, G)
+    st = lib.ssd_decode_step(ctypes.byref(dims), _DTYPES[x.dtype], _ptr(state), _ptr(x), _ptr(dt),
+                             _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(y), _stream(stream))
+    if st != OK:
+        raise SSDError(st, "ssd_decode_step")
+    return y
+
+
+def prefill_host(x, dt, A, B, C, D, chunk: int = 256, device="cuda", stream=None):
+    """End-to-end prefill from host tensors: copies the inputs to the device, runs
+    ssd_prefill and copies y and the final state back into pinned host tensors.
+    Returns (y_host, final_state_host); the copies are ordered on `stream`."""
+    dev = torch.device(device)
+    s = stream or torch.cuda.current_stream(dev)
+    with torch.cuda.stream(s):
+        d_in = [t.to(dev, non_blocking=True) for t in (x, dt, A, B, C, D)]
+        y, fs = prefill(*d_in, chunk=chunk, stream=s)
+        y_h = torch.empty(y.shape, dtype=y.dtype, pin_memory=True)
+        fs_h = torch.empty(fs.shape, dtype=fs.dtype, pin_memory=True)
+        y_h.copy_(y, non_blocking=True)
+        fs_h.copy_(fs, non_blocking=True)
+    return y_h, fs_h

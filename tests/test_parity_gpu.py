@@ -1,0 +1,232 @@
+"""GPU parity: libssd (through its C ABI) against the fp64 CPU oracle on the same seeded
+inputs.  Tolerances: max|y - y_ref| <= 1e-4 RMS(y_ref) for fp32 inputs, <= 2e-2 RMS for
+bf16 inputs (fp32 accumulation, fp32 state); the final state within the same bounds."""
+from dataclasses import replace
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from selective_state_space_10_b200 import inputs
+from helpers import TOL, assert_close, decode_args, rel_err, to_device
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def ssd():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from selective_state_space_10_b200 import ssd as mod
+    return mod
+
+
+def run_prefill(ssd, si, chunk):
+    t = to_device(si)
+    y, fs = ssd.prefill(t["x"], t["dt"], t["A"], t["B"], t["C"], t["D"], chunk=chunk)
+    torch.cuda.synchronize()
+    return y.cpu().numpy(), fs.cpu().numpy()
+
+
+def check_prefill(ssd, si, chunk, what):
+    y, fs = run_prefill(ssd, si, chunk)
+    y_ref, fs_ref = oracle.recurrence(si.x, si.dt, si.A, si.B, si.C, si.D)
+    tol = TOL[si.dtype]
+    ey = assert_close(y, y_ref, tol, f"{what} y")
+    es = assert_close(fs, fs_ref, tol, f"{what} final state")
+    return ey, es
+
+
+# ----------------------------------------------------------------- small cases
+
+def test_tiny_fp32_prefill_then_decode(ssd):
+    """fp32 workload: prefill of 256 tokens, then 16 decode steps of the following tokens;
+    checked against one oracle recurrence over all 272 tokens."""
+    w = inputs.BY_NAME["tiny_fp32"]
+    full = inputs.workload_sequence(w, seqlen=w.seqlen + w.decode_steps)
+    pre = full.token_slice(0, w.seqlen)
+    y, fs = run_prefill(ssd, pre, w.chunk)
+    state = torch.from_numpy(fs).cuda()
+    ys = [y]
+    for k in range(w.decode_steps):
+        tok = to_device(full.token_slice(w.seqlen + k, w.seqlen + k + 1))
+        yk = ssd.decode_step(state, **decode_args(tok))
+        ys.append(yk.cpu().numpy()[:, None])
+    y_all = np.concatenate(ys, axis=1)
+    y_ref, fs_ref = oracle.recurrence(full.x, full.dt, full.A, full.B, full.C, full.D)
+    assert_close(y_all, y_ref, 1e-4, "y over 272 tokens")
+    assert_close(state.cpu().numpy(), fs_ref, 1e-4, "state after 272 tokens")
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("shape", [
+    dict(b=2, L=600, H=4, P=64, N=128, G=1, Q=256),   # several chunks, ragged tail
+    dict(b=1, L=300, H=4, P=64, N=128, G=2, Q=128),   # two groups
+    dict(b=1, L=257, H=3, P=32, N=64, G=1, Q=64),
+    dict(b=2, L=100, H=2, P=100, N=32, G=1, Q=32),    # P not a multiple of 64
+    dict(b=1, L=70, H=2, P=8, N=256, G=1, Q=16),
+    dict(b=1, L=50, H=1, P=1, N=16, G=1, Q=8),
+    dict(b=1, L=130, H=2, P=256, N=128, G=1, Q=64),
+])
+def test_prefill_shapes(ssd, dtype, shape):
+    s = shape
+    si = inputs.sequence(s["b"], s["L"], s["H"], s["P"], s["N"], s["G"], dtype, seed=123)
+    check_prefill(ssd, si, s["Q"], f"{dtype} {s}")
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("chunk", [1, 2, 16, 32, 64, 128, 256])
+def test_chunk_sizes(ssd, dtype, chunk):
+    si = inputs.sequence(1, 333, 2, 64, 128, 1, dtype, seed=7)
+    check_prefill(ssd, si, chunk, f"{dtype} chunk {chunk}")
+
+
+@pytest.mark.parametrize("L", [1, 2, 63, 64, 65, 255, 256, 257])
+def test_lengths_around_chunk(ssd, L):
+    si = inputs.sequence(2, L, 4, 64, 128, 1, "bf16", seed=L)
+    check_prefill(ssd, si, 64 if L < 200 else 256, f"L={L}")
+
+
+def test_empty_sequence_gives_zero_state(ssd):
+    x = torch.empty((2, 0, 4, 64), dtype=torch.bfloat16, device="cuda")
+    dt = torch.empty((2, 0, 4), device="cuda")
+    B = torch.empty((2, 0, 1, 128), dtype=torch.bfloat16, device="cuda")
+    A = -torch.ones(4, device="cuda")
+    D = torch.ones(4, device="cuda")
+    fs = torch.full((2, 4, 64, 128), 7.0, device="cuda")
+    y, fs = ssd.prefill(x, dt, A, B, B, D, chunk=256, final_state=fs)
+    torch.cuda.synchronize()
+    assert y.shape == (2, 0, 4, 64)
+    assert torch.count_nonzero(fs).item() == 0
+
+
+def test_empty_batch(ssd):
+    x = torch.empty((0, 10, 4, 64), dtype=torch.bfloat16, device="cuda")
+    B = torch.empty((0, 10, 1, 128), dtype=torch.bfloat16, device="cuda")
+    y, fs = ssd.prefill(x, torch.empty((0, 10, 4), device="cuda"), -torch.ones(4, device="cuda"), B, B,
+                        torch.ones(4, device="cuda"), chunk=64)
+    assert y.shape == (0, 10, 4, 64) and fs.shape == (0, 4, 64, 128)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_decode_from_random_state(ssd, dtype):
+    w = replace(inputs.BY_NAME["mamba2_2.7b_decode_b256"], batch=3, nheads=8, ngroups=2, dtype=dtype)
+    state0 = inputs.decode_initial_state(w)
+    state = torch.from_numpy(state0).cuda()
+    st_ref = state0.astype(np.float64)
+    for step in range(5):
+        tok = inputs.decode_token(w, step)
+        y = ssd.decode_step(state, **decode_args(to_device(tok)))
+        y_ref, st_ref = oracle.recurrence(tok.x, tok.dt, tok.A, tok.B, tok.C, tok.D, state=st_ref)
+        assert_close(y.cpu().numpy(), y_ref[:, 0], TOL[dtype], f"decode step {step} y")
+    assert_close(state.cpu().numpy(), st_ref, TOL[dtype], "decode state")
+
+
+@pytest.mark.parametrize("N", [16, 32, 64, 256])
+def test_decode_dstates(ssd, N):
+    w = replace(inputs.BY_NAME["mamba2_2.7b_decode_b256"], batch=2, nheads=4, headdim=48, dstate=N)
+    state0 = inputs.decode_initial_state(w)
+    state = torch.from_numpy(state0).cuda()
+    tok = inputs.decode_token(w, 0)
+    y = ssd.decode_step(state, **decode_args(to_device(tok)))
+    y_ref, st_ref = oracle.recurrence(tok.x, tok.dt, tok.A, tok.B, tok.C, tok.D, state=state0)
+    assert_close(y.cpu().numpy(), y_ref[:, 0], 2e-2, f"N={N} y")
+    assert_close(state.cpu().numpy(), st_ref, 2e-2, f"N={N} state")
+
+
+def test_prefill_is_deterministic(ssd):
+    si = inputs.sequence(1, 700, 8, 64, 128, 1, "bf16", seed=3)
+    t = to_device(si)
+    y1, f1 = ssd.prefill(**t, chunk=256)
+    y2, f2 = ssd.prefill(**t, chunk=256)
+    torch.cuda.synchronize()
+    assert torch.equal(y1, y2) and torch.equal(f1, f2)
+
+
+def test_binding_and_abi_errors(ssd):
+    si = inputs.sequence(1, 64, 2, 64, 128, 1, "bf16", seed=1)
+    t = to_device(si)
+    with pytest.raises(ValueError):
+        ssd.prefill(t["x"].float(), t["dt"], t["A"], t["B"], t["C"], t["D"])   # mixed dtypes
+    with pytest.raises(ValueError):
+        ssd.prefill(t["x"], t["dt"].double(), t["A"], t["B"], t["C"], t["D"])
+    # x at a 4-byte offset: the C ABI rejects it (SSD_ERR_INVALID_ARG), nothing launched
+    buf = torch.empty(t["x"].numel() + 2, dtype=torch.bfloat16, device="cuda")
+    xm = buf[2:].view(t["x"].shape)
+    xm.copy_(t["x"])
+    with pytest.raises(ssd.SSDError) as e:
+        ssd.prefill(xm, t["dt"], t["A"], t["B"], t["C"], t["D"])
+    assert e.value.status == ssd.ERR_INVALID_ARG
+    need = ssd.prefill_workspace_size(ssd.dims_of_prefill(t["x"], t["B"]), ssd.BF16, 64)
+    small = torch.empty(need - 256, dtype=torch.uint8, device="cuda")
+    with pytest.raises(ssd.SSDError) as e:
+        ssd.prefill(**t, chunk=64, workspace=small)
+    assert e.value.status == ssd.ERR_WORKSPACE
+
+
+# ----------------------------------------------------------------- full workloads
+
+@pytest.mark.parametrize("name", ["mamba2_130m_prefill", "mamba2_2.7b_prefill"])
+def test_full_prefill_workloads(ssd, name):
+    w = inputs.BY_NAME[name]
+    si = inputs.workload_sequence(w)
+    ey, es = check_prefill(ssd, si, w.chunk, name)
+    print(f"{name}: y err {ey:.2e}, state err {es:.2e} (RMS-relative max)")
+
+
+def test_long_context_prefill_then_decode(ssd):
+    """b=4, L=16384 prefill, then 256 decode steps from its final state, against (i) one
+    GPU prefill of all 16640 tokens (every head) and (ii) the oracle over all 16640
+    tokens on a sample of (batch row, head) pairs."""
+    w = inputs.BY_NAME["mamba2_130m_long_b4"]
+    full = inputs.workload_sequence(w, seqlen=w.seqlen + w.decode_steps)
+    pre = full.token_slice(0, w.seqlen)
+    t_pre = to_device(pre)
+    y_pre, state = ssd.prefill(**t_pre, chunk=w.chunk)
+    del t_pre
+    t_full = to_device(full)
+    ys = []
+    for k in range(w.decode_steps):
+        tok = {kk: (v[:, w.seqlen + k:w.seqlen + k + 1] if v.dim() > 1 else v) for kk, v in t_full.items()}
+        ys.append(ssd.decode_step(state, **decode_args(tok))[:, None])
+    y_split = torch.cat([y_pre] + ys, dim=1)
+    y_one, fs_one = ssd.prefill(**t_full, chunk=w.chunk)
+    torch.cuda.synchronize()
+    y_split, y_one = y_split.cpu().numpy(), y_one.cpu().numpy()
+    assert_close(y_split, y_one, 2e-2, "split vs one prefill y")
+    assert_close(state.cpu().numpy(), fs_one.cpu().numpy(), 2e-2, "split vs one prefill state")
+    rng = np.random.default_rng(0)
+    for bi, h in [(0, 0), (3, 23)] + [tuple(v) for v in rng.integers((0, 0), (4, 24), (2, 2))]:
+        hs = full.head_slice(bi, h)
+        y_ref, fs_ref = oracle.recurrence(hs.x, hs.dt, hs.A, hs.B, hs.C, hs.D)
+        assert_close(y_split[bi:bi + 1, :, h:h + 1], y_ref, 2e-2, f"oracle y (b={bi}, h={h})")
+        assert_close(state.cpu().numpy()[bi:bi + 1, h:h + 1], fs_ref, 2e-2, f"oracle state (b={bi}, h={h})")
+
+
+def test_batched_decode_workload(ssd):
+    """batch 256 x 80 heads, 1024 decode steps from a seeded N(0, 0.1^2) state; y checked
+    against the oracle at steps 0..15, 31, 63, ..., 1023 and the final state, on a sample
+    of (batch row, head) pairs (the oracle runs only those)."""
+    w = inputs.BY_NAME["mamba2_2.7b_decode_b256"]
+    state0 = inputs.decode_initial_state(w)
+    state = torch.from_numpy(state0).cuda()
+    rng = np.random.default_rng(1)
+    pairs = [(0, 0), (255, 79)] + [tuple(v) for v in rng.integers((0, 0), (256, 80), (10, 2))]
+    st_ref = {p: state0[p[0]:p[0] + 1, p[1]:p[1] + 1].astype(np.float64) for p in pairs}
+    checks = set(range(16)) | {31, 63, 127, 255, 511, 1023}
+    worst = 0.0
+    for step in range(w.decode_steps):
+        tok = inputs.decode_token(w, step)
+        y = ssd.decode_step(state, **decode_args(to_device(tok)))
+        for (bi, h) in pairs:
+            hs = tok.head_slice(bi, h)
+            y_ref, st_ref[(bi, h)] = oracle.recurrence(hs.x, hs.dt, hs.A, hs.B, hs.C, hs.D,
+                                                       state=st_ref[(bi, h)], nthreads=1)
+            if step in checks:
+                got = y[bi, h].cpu().numpy()
+                worst = max(worst, assert_close(got, y_ref[0, 0, 0], 2e-2, f"step {step} (b={bi}, h={h})"))
+    st = state.cpu().numpy()
+    for (bi, h) in pairs:
+        assert_close(st[bi, h], st_ref[(bi, h)][0, 0], 2e-2, f"final state (b={bi}, h={h})")
+    print(f"batched decode: worst y err {worst:.2e}")
