@@ -40,7 +40,7 @@
  *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy default
  *     stream): they validate on the host, enqueue kernels and return.  On a validation
  *     error nothing is enqueued.  A launch failure is reported as SSD_ERR_CUDA.  No call
- *     aborts, prints or synchronises.
+ *     aborts or prints, and none but ssd_prefill_device_status synchronises.
  *   - Inputs and outputs must not overlap, except as stated for ssd_decode_step.
  */
 #ifndef LIBSSD_SSD_H_
@@ -149,6 +149,16 @@ SSD_API ssd_status ssd_prefill_timed(const ssd_dims *dims, ssd_dtype dtype, cons
  * order (static storage), or NULL if i is out of range or the arguments are invalid.
  */
 SSD_API const char *ssd_prefill_kernel_name(const ssd_dims *dims, ssd_dtype dtype, int chunk, int i);
+
+/*
+ * Device-side status of the last ssd_prefill that used this workspace: synchronises
+ * `stream`, then reads the workspace's error word.  SSD_ERR_TIMEOUT means a bounded
+ * device-side wait inside the prefill kernels expired (the kernels then stop touching
+ * data and exit; y and final_state are undefined); SSD_OK otherwise.  SSD_ERR_CUDA if
+ * the copy or the synchronisation fails, SSD_ERR_INVALID_ARG for a NULL, misaligned or
+ * too small workspace.  Unlike every other call, this one blocks the host.
+ */
+SSD_API ssd_status ssd_prefill_device_status(const void *workspace, size_t workspace_bytes, ssd_stream_t stream);
 
 /*
  * One cached decode step (O(1) in the sequence length: "Compiler-First State Space

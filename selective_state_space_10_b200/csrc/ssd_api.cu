@@ -57,22 +57,40 @@ bool check_ptr(const void *p, int64_t elems, size_t align) {
   return p != nullptr && aligned(p, align);
 }
 
+enum class Path { kNone, kSimt, kTensorCore };
+
+// Workspace layout of one prefill.  Offset 0 always holds a 256-byte region whose first
+// int is the device-side error word (non-zero after a bounded wait expired).
 struct PrefillPlan {
-  int nc = 0;            // chunks per sequence
-  size_t cum_off = 0;    // float [b][H][nc][Q]
-  size_t states_off = 0; // float [b][nc][H][P][N]
+  Path path = Path::kNone;
+  int nc = 0;             // chunks per sequence
+  size_t cum_off = 0;     // SIMT: float [b][H][nc][Q] in-chunk cumulative decay
+  size_t states_off = 0;  // both: float [b][nc][H][P][N] chunk states (SIMT: replaced by h_prev)
+  size_t cdecay_off = 0;  // tensor cores: float [b][H][nc] total decay of each chunk
+  size_t hprev_off = 0;   // tensor cores: bf16 [b][nc][H][P][N] state entering each chunk
   size_t bytes = 0;
   int launches = 0;
 };
 
-PrefillPlan plan_prefill(const Dims &d, int Q) {
+PrefillPlan plan_prefill(const Dims &d, ssd_dtype dtype, int Q) {
   PrefillPlan pl;
   pl.nc = (int)(((int64_t)d.L + Q - 1) / Q);
   if (d.b == 0 || d.L == 0) return pl;
-  pl.cum_off = 0;
-  pl.states_off = align_up((size_t)d.b * d.H * pl.nc * Q * sizeof(float));
-  pl.bytes = pl.states_off + align_up((size_t)d.b * pl.nc * d.H * (size_t)d.P * d.N * sizeof(float));
-  pl.launches = 4;
+  const size_t nstate = (size_t)d.b * pl.nc * d.H * (size_t)d.P * d.N;
+  if (dtype == SSD_BF16 && ssd::tc_prefill_supported(d, Q)) {
+    pl.path = Path::kTensorCore;
+    pl.states_off = kAlign;
+    pl.cdecay_off = pl.states_off + align_up(nstate * sizeof(float));
+    pl.hprev_off = pl.cdecay_off + align_up((size_t)d.b * d.H * pl.nc * sizeof(float));
+    pl.bytes = pl.hprev_off + align_up(nstate * sizeof(__nv_bfloat16));
+    pl.launches = 3;
+  } else {
+    pl.path = Path::kSimt;
+    pl.cum_off = kAlign;
+    pl.states_off = pl.cum_off + align_up((size_t)d.b * d.H * pl.nc * Q * sizeof(float));
+    pl.bytes = pl.states_off + align_up(nstate * sizeof(float));
+    pl.launches = 4;
+  }
   return pl;
 }
 
@@ -106,6 +124,7 @@ ssd_status run_prefill(const Dims &d, int Q, const PrefillPlan &pl, const T *x, 
 }
 
 const char *const kSimtKernelNames[] = {"dA_cumsum", "chunk_state_simt", "state_passing", "chunk_scan_simt"};
+const char *const kTcKernelNames[] = {"chunk_state_tc", "state_passing_bf16", "chunk_scan_tc"};
 
 }  // namespace
 
@@ -129,14 +148,14 @@ size_t ssd_prefill_workspace_size(const ssd_dims *dims, ssd_dtype dtype, int chu
   Dims d;
   if (check_dims(dims, dtype, true, &d) != SSD_OK) return 0;
   if (!is_pow2(chunk) || chunk > 256) return 0;
-  return plan_prefill(d, chunk).bytes;
+  return plan_prefill(d, dtype, chunk).bytes;
 }
 
 int ssd_prefill_kernel_launches(const ssd_dims *dims, ssd_dtype dtype, int chunk) {
   Dims d;
   if (check_dims(dims, dtype, true, &d) != SSD_OK) return -1;
   if (!is_pow2(chunk) || chunk > 256) return -1;
-  return plan_prefill(d, chunk).launches;
+  return plan_prefill(d, dtype, chunk).launches;
 }
 
 static ssd_status prefill_impl(const ssd_dims *dims, ssd_dtype dtype, const void *x, const float *dt,
@@ -154,7 +173,7 @@ static ssd_status prefill_impl(const ssd_dims *dims, ssd_dtype dtype, const void
     return SSD_ERR_INVALID_ARG;
   const bool any_heads = d.b > 0 && d.L > 0;
   if (!check_ptr(A, any_heads ? d.H : 0, 4) || !check_ptr(D, any_heads ? d.H : 0, 4)) return SSD_ERR_INVALID_ARG;
-  const PrefillPlan pl = plan_prefill(d, chunk);
+  const PrefillPlan pl = plan_prefill(d, dtype, chunk);
   if (timed) {
     if (events == nullptr || num_events < pl.launches + 1) return SSD_ERR_INVALID_ARG;
     for (int i = 0; i < pl.launches + 1; ++i)
@@ -168,6 +187,14 @@ static ssd_status prefill_impl(const ssd_dims *dims, ssd_dtype dtype, const void
   if (d.L == 0) return cuda_status(cudaMemsetAsync(final_state, 0, (size_t)nst * sizeof(float), st));
   char *ws = static_cast<char *>(workspace);
   cudaEvent_t const *ev = timed ? reinterpret_cast<cudaEvent_t const *>(events) : nullptr;
+  cudaError_t e = cudaMemsetAsync(ws, 0, sizeof(int), st);  // device error word
+  if (e != cudaSuccess) return SSD_ERR_CUDA;
+  if (pl.path == Path::kTensorCore)
+    return cuda_status(ssd::launch_tc_prefill(
+        static_cast<const __nv_bfloat16 *>(x), dt, A, static_cast<const __nv_bfloat16 *>(B),
+        static_cast<const __nv_bfloat16 *>(C), D, y, final_state, reinterpret_cast<float *>(ws + pl.states_off),
+        reinterpret_cast<float *>(ws + pl.cdecay_off), reinterpret_cast<__nv_bfloat16 *>(ws + pl.hprev_off),
+        reinterpret_cast<int *>(ws), d, chunk, pl.nc, st, ev));
   if (dtype == SSD_F32)
     return run_prefill<float>(d, chunk, pl, static_cast<const float *>(x), dt, A, static_cast<const float *>(B),
                               static_cast<const float *>(C), D, y, final_state, ws, st, ev);
@@ -194,9 +221,18 @@ ssd_status ssd_prefill_timed(const ssd_dims *dims, ssd_dtype dtype, const void *
 const char *ssd_prefill_kernel_name(const ssd_dims *dims, ssd_dtype dtype, int chunk, int i) {
   Dims d;
   if (check_dims(dims, dtype, true, &d) != SSD_OK || !is_pow2(chunk) || chunk > 256) return nullptr;
-  const PrefillPlan pl = plan_prefill(d, chunk);
+  const PrefillPlan pl = plan_prefill(d, dtype, chunk);
   if (i < 0 || i >= pl.launches) return nullptr;
-  return kSimtKernelNames[i];
+  return pl.path == Path::kTensorCore ? kTcKernelNames[i] : kSimtKernelNames[i];
+}
+
+ssd_status ssd_prefill_device_status(const void *workspace, size_t workspace_bytes, ssd_stream_t stream) {
+  if (workspace == nullptr || workspace_bytes < sizeof(int) || !aligned(workspace, 16)) return SSD_ERR_INVALID_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  int word = 0;
+  if (cudaMemcpyAsync(&word, workspace, sizeof(int), cudaMemcpyDeviceToHost, st) != cudaSuccess) return SSD_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return SSD_ERR_CUDA;
+  return word == 0 ? SSD_OK : SSD_ERR_TIMEOUT;
 }
 
 ssd_status ssd_decode_step(const ssd_dims *dims, ssd_dtype dtype, float *state, const void *x, const float *dt,

@@ -33,7 +33,7 @@ class Dims(ctypes.Structure):
 # Every symbol include/ssd.h declares.
 EXPORTS = ("ssd_status_string", "ssd_version", "ssd_prefill_workspace_size",
            "ssd_prefill_kernel_launches", "ssd_prefill", "ssd_prefill_timed",
-           "ssd_prefill_kernel_name", "ssd_decode_step")
+           "ssd_prefill_kernel_name", "ssd_prefill_device_status", "ssd_decode_step")
 
 
 def _load():
@@ -58,6 +58,8 @@ def _load():
     lib.ssd_prefill_timed.restype = ci
     lib.ssd_prefill_kernel_name.argtypes = [dp, ci, ci, ci]
     lib.ssd_prefill_kernel_name.restype = ctypes.c_char_p
+    lib.ssd_prefill_device_status.argtypes = [vp, sz, vp]
+    lib.ssd_prefill_device_status.restype = ci
     lib.ssd_decode_step.argtypes = [dp, ci, fp, vp, fp, fp, vp, vp, fp, fp, vp]
     lib.ssd_decode_step.restype = ci
     return lib
@@ -164,6 +166,13 @@ def prefill(x, dt, A, B, C, D, chunk: int = 256, y=None, final_state=None, works
     if st != OK:
         raise SSDError(st, "ssd_prefill")
     return y, final_state
+
+
+def prefill_device_status(workspace, stream=None) -> int:
+    """Blocks until `stream` is idle, then returns the status word the prefill kernels
+    left in `workspace` (OK, or ERR_TIMEOUT if a bounded device-side wait expired)."""
+    return lib.ssd_prefill_device_status(_ptr(workspace), workspace.numel() * workspace.element_size(),
+                                         _stream(stream))
 
 
 def decode_step(state, x, dt, A, B, C, D, y=None, stream=None) -> torch.Tensor:
