@@ -35,6 +35,7 @@
 // touching further data.
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <stddef.h>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -51,24 +52,26 @@ constexpr int TN = 128;   // d_state handled by the tensor-core path
 
 // ============================================================================ K1
 constexpr int K1_SLOTS = 2;
-constexpr int K1_THREADS = 320;  // warp 0 TMA, warp 1 MMA, warps 2-5 scale, warps 6-9 epilogue
+constexpr int K1_CUMBUF = 3;
+constexpr int K1_THREADS = 352;  // warp 0 TMA, 1 MMA, 2-5 scale, 6-9 epilogue, 10 decay weights
 
 struct K1Smem {
   // offsets from the 1024-aligned base
   static constexpr uint32_t bm = 0;  // B chunk: 2 x [Q][128 B]
   // slot s: x (scaled in place to the bf16 high part) at x(), the bf16 remainder at lo()
-  static constexpr uint32_t x(int Q, int s) { return 2u * Q * 128u + (uint32_t)s * 2u * Q * 128u; }
-  static constexpr uint32_t lo(int Q, int s) { return x(Q, s) + (uint32_t)Q * 128u; }
-  static constexpr uint32_t misc(int Q) { return 2u * Q * 128u + K1_SLOTS * 2u * Q * 128u; }
+  __host__ __device__ static constexpr uint32_t x(int Q, int s) { return 2u * Q * 128u + (uint32_t)s * 2u * Q * 128u; }
+  __host__ __device__ static constexpr uint32_t lo(int Q, int s) { return x(Q, s) + (uint32_t)Q * 128u; }
+  __host__ __device__ static constexpr uint32_t misc(int Q) { return 2u * Q * 128u + K1_SLOTS * 2u * Q * 128u; }
 };
 
 struct K1Misc {
   uint64_t b_full;
   uint64_t x_full[K1_SLOTS], scaled[K1_SLOTS], x_free[K1_SLOTS];
   uint64_t acc_full[2], acc_free[2];
+  uint64_t w_full[K1_CUMBUF], w_free[K1_CUMBUF];
   uint32_t tmem;
   int abort_flag;
-  float w[2][256];  // decay weights of the current head (double-buffered by head parity)
+  float w[K1_CUMBUF][256];  // decay weights exp(cum_end - cum_t) dt_t of upcoming heads
 };
 
 __global__ void __launch_bounds__(K1_THREADS, 1)
@@ -103,6 +106,10 @@ k_chunk_state_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
     for (int a = 0; a < 2; ++a) {
       mbar_init(&ms->acc_full[a], 1);
       mbar_init(&ms->acc_free[a], 1);
+    }
+    for (int i = 0; i < K1_CUMBUF; ++i) {
+      mbar_init(&ms->w_full[i], 1);
+      mbar_init(&ms->w_free[i], 1);
     }
     ms->abort_flag = 0;
     mbar_fence_init();
@@ -171,60 +178,39 @@ k_chunk_state_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
     // ------------------------------------------------------------- scale warps (128 threads)
     const int tid = threadIdx.x - 64;
     for (int k = 0; k < nh; ++k) {
-      const int s = k % K1_SLOTS, hp = k & 1, h = h0 + k;
-      if (warp == 2 && !*abort_flag) {
-        // in-chunk cumulative log2-decay, then w_t = exp(cum_end - cum_t) dt_t
-        const float a2 = A[h] * kLog2e;
-        const int per = Q / 32;
-        float c2[8], dtv[8];
-        float run = 0.f;
-        for (int j = 0; j < per; ++j) {
-          const int t = lane * per + j;
-          dtv[j] = (t < valid) ? dt[((size_t)bi * d.L + t0 + t) * d.H + h] : 0.f;
-          run += dtv[j] * a2;
-          c2[j] = run;
-        }
-        float incl = run;
+      const int s = k % K1_SLOTS, wb = k % K1_CUMBUF;
+      bool ok = mbar_wait(&ms->w_full[wb], (k / K1_CUMBUF) & 1, abort_flag, err);
+      ok = ok && mbar_wait(&ms->x_full[s], (k / K1_SLOTS) & 1, abort_flag, err);
+      if (ok) {
+        const uint32_t xs = smem_u32(base + K1Smem::x(Q, s));
+        const uint32_t ls = smem_u32(base + K1Smem::lo(Q, s));
+        const float *wv_row = ms->w[wb];
+        for (int unit = tid; unit < Q * 8; unit += 128) {
+          const float wv = wv_row[unit >> 3];
+          const uint32_t off = (uint32_t)unit * 16u;  // rows are 128 B: unit*16 = row*128 + chunk*16
+          const uint4 v = ld_shared_v4(xs + off);
+          const uint32_t in[4] = {v.x, v.y, v.z, v.w};
+          uint32_t hi[4], rem[4];
 #pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const float v = __shfl_up_sync(0xffffffffu, incl, o);
-          if (lane >= o) incl += v;
+          for (int q = 0; q < 4; ++q) {
+            const float a0 = __uint_as_float(in[q] << 16) * wv;  // exact x * w in fp32
+            const float a1 = __uint_as_float(in[q] & 0xffff0000u) * wv;
+            hi[q] = pack_bf16x2(a0, a1);
+            const float h0 = __uint_as_float(hi[q] << 16), h1 = __uint_as_float(hi[q] & 0xffff0000u);
+            rem[q] = pack_bf16x2(a0 - h0, a1 - h1);
+          }
+          st_shared_v4(xs + off, hi[0], hi[1], hi[2], hi[3]);
+          st_shared_v4(ls + off, rem[0], rem[1], rem[2], rem[3]);
         }
-        const float excl = incl - run;
-        const float cend = __shfl_sync(0xffffffffu, incl, 31);
-        for (int j = 0; j < per; ++j) ms->w[hp][lane * per + j] = ex2(cend - (c2[j] + excl)) * dtv[j];
-        if (lane == 0) cdecay[((size_t)bi * d.H + h) * nc + c] = ex2(cend);
-      }
-      named_barrier(1, 128);
-      if (!mbar_wait(&ms->x_full[s], (k / K1_SLOTS) & 1, abort_flag, err)) {
-        named_barrier(1, 128);
-        continue;
-      }
-      const uint32_t xs = smem_u32(base + K1Smem::x(Q, s));
-      const uint32_t ls = smem_u32(base + K1Smem::lo(Q, s));
-      for (int unit = tid; unit < Q * 8; unit += 128) {
-        const int row = unit >> 3;
-        const float wv = ms->w[hp][row];
-        const uint32_t off = (uint32_t)unit * 16u;  // rows are 128 B: unit*16 = row*128 + chunk*16
-        const uint4 v = ld_shared_v4(xs + off);
-        const uint32_t in[4] = {v.x, v.y, v.z, v.w};
-        uint32_t hi[4], rem[4];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const float a0 = __uint_as_float(in[q] << 16) * wv;          // exact x * w in fp32
-          const float a1 = __uint_as_float(in[q] & 0xffff0000u) * wv;
-          hi[q] = pack_bf16x2(a0, a1);
-          const float h0 = __uint_as_float(hi[q] << 16), h1 = __uint_as_float(hi[q] & 0xffff0000u);
-          rem[q] = pack_bf16x2(a0 - h0, a1 - h1);
-        }
-        st_shared_v4(xs + off, hi[0], hi[1], hi[2], hi[3]);
-        st_shared_v4(ls + off, rem[0], rem[1], rem[2], rem[3]);
       }
       fence_proxy_async_smem();
       named_barrier(1, 128);
-      if (tid == 0) mbar_arrive(&ms->scaled[s]);
+      if (tid == 0 && ok) {
+        mbar_arrive(&ms->scaled[s]);
+        mbar_arrive(&ms->w_free[wb]);
+      }
     }
-  } else {
+  } else if (warp < 10) {
     // ------------------------------------------------------------- epilogue warps (128 threads)
     const int q = warp & 3;
     const int n = q * 32 + lane;  // d_state row of the accumulator
@@ -248,6 +234,39 @@ k_chunk_state_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
       named_barrier(2, 128);
       if (tid == 0) mbar_arrive(&ms->acc_free[a]);
     }
+  } else {
+    // ------------------------------------------------------------- decay-weight warp
+    // w_t = exp(cum_end - cum_t) dt_t for each upcoming head (ring of K1_CUMBUF), and the
+    // chunk's total decay exp(cum_end) for the state-passing kernel.
+    const int per = Q / 32;
+    for (int k = 0; k < nh; ++k) {
+      const int wb = k % K1_CUMBUF, h = h0 + k;
+      if (k >= K1_CUMBUF && !mbar_wait(&ms->w_free[wb], ((k / K1_CUMBUF) - 1) & 1, abort_flag, err)) break;
+      const float a2 = A[h] * kLog2e;
+      float c2[8], dtv[8];
+      float run = 0.f;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int t = lane * per + j;
+        dtv[j] = (j < per && t < valid) ? dt[((size_t)bi * d.L + t0 + t) * d.H + h] : 0.f;
+        run += dtv[j] * a2;
+        c2[j] = run;
+      }
+      float incl = run;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const float v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+      }
+      const float excl = incl - run;
+      const float cend = __shfl_sync(0xffffffffu, incl, 31);
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        if (j < per) ms->w[wb][lane * per + j] = ex2(cend - (c2[j] + excl)) * dtv[j];
+      if (lane == 0) cdecay[((size_t)bi * d.H + h) * nc + c] = ex2(cend);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ms->w_full[wb]);
+    }
   }
 
   tc_fence_before();
@@ -259,75 +278,112 @@ k_chunk_state_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
 }
 
 // ============================================================================ K2
-// grid (b * H, P*N / 8 / 256), block 256: 8 consecutive state elements per thread.
+// grid (b * H, ceil(P*N/4 / 256)), block 256: one float4 of the state per thread.  The
+// chunk states of 8 chunks are loaded before the sequential update so that their
+// latencies overlap; the state entering chunk c is stored in bf16, the final state in fp32.
+constexpr int K2_BATCH = 8;
+
 __global__ void __launch_bounds__(256)
 k_state_passing_bf16(const float *__restrict__ states, const float *__restrict__ cdecay,
                      __nv_bfloat16 *__restrict__ hprev, float *__restrict__ final_state, Dims d, int nc) {
-  const int PN = d.P * d.N;
-  const int e = (blockIdx.y * blockDim.x + threadIdx.x) * 8;
-  if (e >= PN) return;
+  const int PN4 = d.P * d.N / 4;
+  const int e4 = blockIdx.y * blockDim.x + threadIdx.x;
+  if (e4 >= PN4) return;
   const int h = blockIdx.x % d.H, bi = blockIdx.x / d.H;
-  const size_t cstride = (size_t)d.H * PN;
-  const size_t off0 = ((size_t)bi * nc * d.H + h) * PN + e;
+  const size_t cstride = (size_t)d.H * PN4;  // float4s between consecutive chunks
+  const size_t off0 = ((size_t)bi * nc * d.H + h) * PN4 + e4;
+  const float4 *sp = reinterpret_cast<const float4 *>(states) + off0;
+  uint2 *hp = reinterpret_cast<uint2 *>(hprev) + off0;
   const float *dec = cdecay + ((size_t)bi * d.H + h) * nc;
-  float hs[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-  float4 s0 = *reinterpret_cast<const float4 *>(states + off0);
-  float4 s1 = *reinterpret_cast<const float4 *>(states + off0 + 4);
-  for (int c = 0; c < nc; ++c) {
-    const size_t off = off0 + (size_t)c * cstride;
-    float4 n0 = make_float4(0.f, 0.f, 0.f, 0.f), n1 = n0;
-    if (c + 1 < nc) {
-      n0 = *reinterpret_cast<const float4 *>(states + off + cstride);
-      n1 = *reinterpret_cast<const float4 *>(states + off + cstride + 4);
-    }
-    uint4 packed;
-    packed.x = sm100::pack_bf16x2(hs[0], hs[1]);
-    packed.y = sm100::pack_bf16x2(hs[2], hs[3]);
-    packed.z = sm100::pack_bf16x2(hs[4], hs[5]);
-    packed.w = sm100::pack_bf16x2(hs[6], hs[7]);
-    *reinterpret_cast<uint4 *>(hprev + off) = packed;  // state entering chunk c
-    const float dc = dec[c];
-    const float sv[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+  float4 hs = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int c0 = 0; c0 < nc; c0 += K2_BATCH) {
+    float4 sv[K2_BATCH];
+    float dc[K2_BATCH];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) hs[j] = fmaf(dc, hs[j], sv[j]);
-    s0 = n0;
-    s1 = n1;
+    for (int j = 0; j < K2_BATCH; ++j)
+      if (c0 + j < nc) {
+        sv[j] = __ldcs(sp + (size_t)(c0 + j) * cstride);
+        dc[j] = dec[c0 + j];
+      }
+#pragma unroll
+    for (int j = 0; j < K2_BATCH; ++j)
+      if (c0 + j < nc) {
+        hp[(size_t)(c0 + j) * cstride] = make_uint2(sm100::pack_bf16x2(hs.x, hs.y), sm100::pack_bf16x2(hs.z, hs.w));
+        hs.x = fmaf(dc[j], hs.x, sv[j].x);
+        hs.y = fmaf(dc[j], hs.y, sv[j].y);
+        hs.z = fmaf(dc[j], hs.z, sv[j].z);
+        hs.w = fmaf(dc[j], hs.w, sv[j].w);
+      }
   }
-  float *fo = final_state + ((size_t)bi * d.H + h) * PN + e;
-  *reinterpret_cast<float4 *>(fo) = make_float4(hs[0], hs[1], hs[2], hs[3]);
-  *reinterpret_cast<float4 *>(fo + 4) = make_float4(hs[4], hs[5], hs[6], hs[7]);
+  reinterpret_cast<float4 *>(final_state)[((size_t)bi * d.H + h) * PN4 + e4] = hs;
 }
 
 // ============================================================================ K3
-constexpr int K3_THREADS = 448;  // warp 0 TMA, 1 MMA, 2-9 W builders, 10-13 output
+// Per CTA: one 128-row token tile (chunk-relative rows 128*ti ..) of one chunk, for a block
+// of heads of one group.  G = C_tile B_chunk^T (fp32, TMEM) is computed once.
+//
+// Decay factorisation.  For a row t and a source token s <= t of the chunk, the decay is
+// 2^(c2_t - c2_s) with c2 the in-chunk cumulative log2-decay of the head.  With the
+// reference token r = 128*ti - 1 (c2_r = 0 for ti = 0: the chunk start) it splits into a
+// row factor u_t = 2^(c2_t - c2_r) and a column factor v_s = 2^(c2_r - c2_s) dt_s.  Hence
+//     sum_s W_ts x_s = u_t * sum_s (G o mask)_ts (v_s x_s),
+// where G o mask (causal) does not depend on the head: it is converted to bf16 once per
+// CTA (W_base), and each head only scales the rows of its x tile by v_s.  This is exact
+// algebra; it is used when the tile's decay range |c2_r - c2_last| is below 100 (then
+// every factor lies in [2^-100, 2^100] and all intermediates stay normal fp32).  Heads
+// with a steeper tile ("steep" heads) build their own W with per-32-token references
+// instead, as a slower exact fallback.
+constexpr int K3_THREADS = 480;  // warp 0 TMA, 1 MMA, 2-9 W/x scaling, 10-13 output, 14 decay tables
 constexpr int K3_CUMBUF = 3;
+constexpr float kSteepLog2 = 100.f;
 
 struct K3Smem {
-  static constexpr uint32_t cm = 0;              // C tile: 2 K-atoms x [128][128 B]      32 KB
-  static constexpr uint32_t bw = 32768;          // B rows (for G), then W blocks          64 KB
-  static constexpr uint32_t x(int s) { return 98304u + (uint32_t)s * 32768u; }  // 2 x 32 KB
-  static constexpr uint32_t hs(int s) { return 163840u + (uint32_t)s * 16384u; } // 2 x 16 KB
+  static constexpr uint32_t cm = 0;      // C tile: 2 K-atoms x [128][128 B]                          32 KB
+  static constexpr uint32_t bw = 32768;  // B rows (for G), then W (W_base or a steep head's W)       64 KB
+  // x tiles: nblk blocks of [128 rows][128 B]; after the head's MMAs, y staging (2 x [128][128 B])
+  __host__ __device__ static constexpr uint32_t x(int s) { return 98304u + (uint32_t)s * 32768u; }  // 2 x 32 KB
+  __host__ __device__ static constexpr uint32_t hs(int s) { return 163840u + (uint32_t)s * 16384u; } // 2 x 16 KB
   static constexpr uint32_t misc = 196608u;
 };
 
 struct K3Misc {
-  uint64_t cb_full, g_full, w_full, w_free;
-  uint64_t x_full[2], x_free[2], acc_full[2], acc_free[2];
+  uint64_t cb_full, g_full;
+  uint64_t x_full[2], ops_ready[2], x_free[2], acc_full[2], acc_free[2];
   uint64_t cum_full[K3_CUMBUF], cum_free[K3_CUMBUF];
   uint32_t tmem;
   int abort_flag;
-  float c2[K3_CUMBUF][256];   // in-chunk cumulative log2-decay
-  float dts[K3_CUMBUF][256];  // dt of each token of the chunk (0 past the end)
-  float vf[K3_CUMBUF][128];   // exp(cum_r - cum_s) dt_s for s in the block before the row tile
+  int steep[K3_CUMBUF];
+  float c2ref[K3_CUMBUF];
+  // tables are read with 16-byte vector loads: keep every row 16-byte aligned
+  alignas(16) float c2[K3_CUMBUF][256];   // in-chunk cumulative log2-decay
+  alignas(16) float dts[K3_CUMBUF][256];  // dt of each token of the chunk (0 past the end)
+  alignas(16) float v[K3_CUMBUF][256];    // 2^(c2_r - c2_s) dt_s, s < 128 * (ti + 1)
+  // steep heads only (per-32-token references):
+  alignas(16) float vo[K3_CUMBUF][256];   // ref = last token of s's 32-token group
+  alignas(16) float vd[K3_CUMBUF][256];   // ref = first token of s's 32-token group
 };
+static_assert(offsetof(K3Misc, c2) % 16 == 0 && offsetof(K3Misc, v) % 16 == 0 && offsetof(K3Misc, vo) % 16 == 0 &&
+                  offsetof(K3Misc, vd) % 16 == 0,
+              "decay tables must be 16-byte aligned");
+static_assert(K3Smem::misc % 16 == 0, "K3Misc must start 16-byte aligned");
 
 constexpr size_t kK3SmemBytes = 1024 + K3Smem::misc + sizeof(K3Misc);
+
+// Writes 32 bf16 (packed pairs) into a K-major 128B-swizzled row: chunks cc0..cc0+3.
+__device__ __forceinline__ void st_row_bf16(uint32_t row_addr, int row, int cc0, const float *g) {
+#pragma unroll
+  for (int cc = 0; cc < 4; ++cc)
+    st_shared_v4(row_addr + (((cc0 + cc) ^ (row & 7)) << 4), pack_bf16x2(g[8 * cc + 0], g[8 * cc + 1]),
+                 pack_bf16x2(g[8 * cc + 2], g[8 * cc + 3]), pack_bf16x2(g[8 * cc + 4], g[8 * cc + 5]),
+                 pack_bf16x2(g[8 * cc + 6], g[8 * cc + 7]));
+}
 
 __global__ void __launch_bounds__(K3_THREADS, 1)
 k_chunk_scan_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_C,
                 const __grid_constant__ CUtensorMap tm_B, const __grid_constant__ CUtensorMap tm_h,
-                const float *__restrict__ dt, const float *__restrict__ A, const float *__restrict__ D,
-                float *__restrict__ y, int *err, Dims d, int Q, int nc, int kb, int nhb) {
+                const __grid_constant__ CUtensorMap tm_y, const __nv_bfloat16 *__restrict__ x,
+                const float *__restrict__ dt, const float *__restrict__ A, const float *__restrict__ D, int *err,
+                Dims d, int Q, int nc, int kb, int nhb) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   K3Misc *ms = reinterpret_cast<K3Misc *>(base + K3Smem::misc);
@@ -353,17 +409,16 @@ k_chunk_scan_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
   if (threadIdx.x == 0) {
     mbar_init(&ms->cb_full, 1);
     mbar_init(&ms->g_full, 1);
-    mbar_init(&ms->w_full, 1);
-    mbar_init(&ms->w_free, 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(&ms->x_full[s], 1);
-      mbar_init(&ms->x_free[s], 2);  // MMA commit + output warps
+      mbar_init(&ms->ops_ready[s], 1);
+      mbar_init(&ms->x_free[s], 2);  // MMA commit + output (y staged out of the slot)
       mbar_init(&ms->acc_full[s], 1);
       mbar_init(&ms->acc_free[s], 1);
     }
     for (int s = 0; s < K3_CUMBUF; ++s) {
       mbar_init(&ms->cum_full[s], 1);
-      mbar_init(&ms->cum_free[s], 1);
+      mbar_init(&ms->cum_free[s], 2);  // x/W warps + output warps
     }
     ms->abort_flag = 0;
     mbar_fence_init();
@@ -386,6 +441,7 @@ k_chunk_scan_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
       tma_prefetch_desc(&tm_C);
       tma_prefetch_desc(&tm_B);
       tma_prefetch_desc(&tm_h);
+      tma_prefetch_desc(&tm_y);
       mbar_arrive_expect_tx(&ms->cb_full, 32768u + (uint32_t)nblk * 32768u);
       for (int kn = 0; kn < 2; ++kn)
         tma_load_3d(base + K3Smem::cm + kn * 16384u, &tm_C, &ms->cb_full, g * TN + 64 * kn, t0 + 128 * ti, bi);
@@ -439,7 +495,7 @@ k_chunk_scan_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
           const uint64_t bd = smem_desc_sw128(hsa + (ks >> 2) * 8192u + (ks & 3) * 32u, 16u, 1024u);
           mma_bf16(acc, ad, bd, id_inter, ks > 0 ? 1u : 0u);
         }
-        if (!mbar_wait(&ms->w_full, k & 1, abort_flag, err)) break;
+        if (!mbar_wait(&ms->ops_ready[s], u & 1, abort_flag, err)) break;
         tc_fence_after();
         const uint32_t xa = smem_u32(base + K3Smem::x(s));
         for (int j = 0; j < nblk; ++j)
@@ -449,107 +505,121 @@ k_chunk_scan_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
             mma_bf16(acc + 64, ad, bd, id_intra, (j > 0 || ks > 0) ? 1u : 0u);
           }
         mma_commit(&ms->acc_full[s]);
-        mma_commit(&ms->w_free);
         mma_commit(&ms->x_free[s]);
       }
     }
     __syncwarp();
   } else if (warp < 10) {
-    // ------------------------------------------------------------- W builders (256 threads)
+    // ------------------------------------------------------------- W build and x scaling (256 threads)
+    // W builds: thread (q, ch, lane) owns row tl = 32q + lane, columns [64ch, 64ch + 64) of
+    // each source block (the warp's rows are the 32-token group q of the tile).
     const int q = warp & 3, ch = (warp - 2) >> 2;
-    const int tl = q * 32 + lane;        // row of the tile (TMEM lane)
+    const int tl = q * 32 + lane;
     const int tid = threadIdx.x - 64;
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
-    const int r = 128 * ti - 1;          // last token before the row tile
-    bool g_ready = false;
+    const int t = 128 * ti + tl;  // chunk-relative row
+    const int r = 128 * ti - 1;   // reference token (tile start)
+    bool g_ready = false, w_is_base = false;
     for (int k = 0; k < nh; ++k) {
-      const int cb = k % K3_CUMBUF, h = h0 + k;
-      // (1) cumulative decay of head h for the whole chunk, by one warp
-      if (warp == 2) {
-        bool ok = true;
-        if (k >= K3_CUMBUF) ok = mbar_wait(&ms->cum_free[cb], ((k / K3_CUMBUF) - 1) & 1, abort_flag, err);
-        if (ok && !*abort_flag) {
-          const float a2 = A[h] * kLog2e;
-          const int per = Q / 32;
-          float c2[8], dtv[8];
-          float run = 0.f;
-          for (int j = 0; j < per; ++j) {
-            const int t = lane * per + j;
-            dtv[j] = (t < valid) ? dt[((size_t)bi * d.L + t0 + t) * d.H + h] : 0.f;
-            run += dtv[j] * a2;
-            c2[j] = run;
-          }
-          float incl = run;
+      const int cb = k % K3_CUMBUF, s = k & 1;
+      bool ok = mbar_wait(&ms->cum_full[cb], (k / K3_CUMBUF) & 1, abort_flag, err);
+      const bool steep = ok && ms->steep[cb];
+      if (ok && (steep || !w_is_base)) {
+        // (re)build W: wait for every earlier MMA that reads the W region (the last is head k-1's)
+        if (k >= 1) ok = mbar_wait(&ms->x_free[(k - 1) & 1], ((k - 1) >> 1) & 1, abort_flag, err);
+        if (ok && !g_ready) ok = g_ready = mbar_wait(&ms->g_full, 0, abort_flag, err);
+        tc_fence_after();
+        if (ok) {
+          const float *c2 = ms->c2[cb];
+          const float c2t = c2[t];
+          for (int j = 0; j < nblk; ++j) {
+            const uint32_t wrow = smem_u32(base + K3Smem::bw) + j * 32768u + ch * 16384u + (uint32_t)tl * 128u;
+            const int grp0 = 2 * ch;  // first of my two 32-column groups within block j
+            if (j == ti && grp0 > q) {  // both groups strictly right of the diagonal
 #pragma unroll
-          for (int o = 1; o < 32; o <<= 1) {
-            const float v = __shfl_up_sync(0xffffffffu, incl, o);
-            if (lane >= o) incl += v;
+              for (int cc = 0; cc < 8; ++cc) st_shared_v4(wrow + ((cc ^ (tl & 7)) << 4), 0u, 0u, 0u, 0u);
+              continue;
+            }
+            float gv[64];
+            tmem_ld32(tmem + lane_off + TM_G + (uint32_t)(128 * j + 64 * ch), *reinterpret_cast<float(*)[32]>(&gv[0]));
+            tmem_ld32(tmem + lane_off + TM_G + (uint32_t)(128 * j + 64 * ch + 32),
+                      *reinterpret_cast<float(*)[32]>(&gv[32]));
+            tmem_ld_wait();
+#pragma unroll
+            for (int gs = 0; gs < 2; ++gs) {
+              const int grp = grp0 + gs;
+              const int col0 = 128 * j + 32 * grp;  // chunk-relative first column
+              float *gg = &gv[32 * gs];
+              if (j == ti && grp > q) {
+#pragma unroll
+                for (int e = 0; e < 32; ++e) gg[e] = 0.f;
+              } else if (!steep) {
+                // W_base = G o causal mask
+                if (j == ti && grp == q) {
+#pragma unroll
+                  for (int e = 0; e < 32; ++e) gg[e] = (col0 + e <= t) ? gg[e] : 0.f;
+                }
+              } else if (j < ti) {
+                const float u = ex2(c2t - c2[r]);
+                const float *vf = ms->v[cb] + col0;  // reference r: the column factors of x scaling
+#pragma unroll
+                for (int e = 0; e < 32; ++e) gg[e] *= vf[e] * u;
+              } else if (grp < q) {
+                const float u = ex2(c2t - c2[col0 + 31]);
+                const float *vo = ms->vo[cb] + col0;
+#pragma unroll
+                for (int e = 0; e < 32; ++e) gg[e] *= vo[e] * u;
+              } else {  // grp == q: own 32-token group, masked
+                const float range = c2[col0] - c2[col0 + 31];
+                if (fabsf(range) < kSteepLog2) {
+                  const float u = ex2(c2t - c2[col0]);
+                  const float *vd = ms->vd[cb] + col0;
+#pragma unroll
+                  for (int e = 0; e < 32; ++e) gg[e] = (col0 + e <= t) ? gg[e] * (vd[e] * u) : 0.f;
+                } else {  // decay too steep even inside the group: one exp per element
+                  const float *dts = ms->dts[cb];
+#pragma unroll
+                  for (int e = 0; e < 32; ++e) {
+                    const int sidx = col0 + e;
+                    gg[e] = (sidx <= t) ? gg[e] * ex2(c2t - c2[sidx]) * dts[sidx] : 0.f;
+                  }
+                }
+              }
+            }
+            st_row_bf16(wrow, tl, 0, &gv[0]);
+            st_row_bf16(wrow, tl, 4, &gv[32]);
           }
-          const float excl = incl - run;
-          for (int j = 0; j < per; ++j) {
-            ms->c2[cb][lane * per + j] = c2[j] + excl;
-            ms->dts[cb][lane * per + j] = dtv[j];
-          }
-          __syncwarp();
-          if (ti > 0) {
-            const float c2r = ms->c2[cb][r];
-            for (int sidx = lane; sidx < 128 * ti; sidx += 32)
-              ms->vf[cb][sidx] = ex2(c2r - ms->c2[cb][sidx]) * ms->dts[cb][sidx];
-          }
+          w_is_base = !steep;
         }
       }
-      named_barrier(1, 256);
-      if (tid == 0) mbar_arrive(&ms->cum_full[cb]);
-      // (2) wait until G is ready and the previous head's MMAs no longer read W
-      if (!g_ready) {
-        g_ready = mbar_wait(&ms->g_full, 0, abort_flag, err);
-      }
-      bool ok = g_ready;
-      if (ok && k >= 1) ok = mbar_wait(&ms->w_free, (k - 1) & 1, abort_flag, err);
-      tc_fence_after();
-      if (ok) {
-        const float *c2 = ms->c2[cb];
-        const float *dts = ms->dts[cb];
-        const int t = 128 * ti + tl;          // chunk-relative row
-        const float c2t = c2[t];
-        for (int j = 0; j < nblk; ++j) {
-          const uint32_t wrow = smem_u32(base + K3Smem::bw) + j * 32768u + ch * 16384u + (uint32_t)tl * 128u;
-          const int s0 = 128 * j + 64 * ch;   // first source token of my 64 columns
-          if (j == ti && q * 32 + 31 < 64 * ch) {
-            // whole warp strictly above the diagonal: zeros
+      // scale the rows of this head's x tile by v_s (not for steep heads: their W holds the decay)
+      ok = ok && mbar_wait(&ms->x_full[s], (k >> 1) & 1, abort_flag, err);
+      if (ok && !steep) {
+        const uint32_t xs = smem_u32(base + K3Smem::x(s));
+        const float *vt = ms->v[cb];
+        const int units = nblk * 128 * 8;  // 16-byte units: row = unit / 8 (rows of 128 B)
+#pragma unroll 4
+        for (int unit = tid; unit < units; unit += 256) {
+          const float vv = vt[unit >> 3];
+          const uint32_t addr = xs + (uint32_t)unit * 16u;
+          const uint4 in = ld_shared_v4(addr);
+          const uint32_t w4[4] = {in.x, in.y, in.z, in.w};
+          uint32_t o4[4];
 #pragma unroll
-            for (int cc = 0; cc < 8; ++cc) st_shared_v4(wrow + ((cc ^ (tl & 7)) << 4), 0u, 0u, 0u, 0u);
-            continue;
-          }
-          float gv[64];
-          tmem_ld32(tmem + lane_off + TM_G + (uint32_t)s0, *reinterpret_cast<float(*)[32]>(&gv[0]));
-          tmem_ld32(tmem + lane_off + TM_G + (uint32_t)s0 + 32u, *reinterpret_cast<float(*)[32]>(&gv[32]));
-          tmem_ld_wait();
-          if (j < ti) {
-            const float ut = ex2(c2t - c2[r]);
-            const float *vf = ms->vf[cb] + s0;
-#pragma unroll
-            for (int e = 0; e < 64; ++e) gv[e] = gv[e] * vf[e] * ut;
-          } else {
-#pragma unroll
-            for (int e = 0; e < 64; ++e) {
-              const int sidx = s0 + e;
-              gv[e] = (sidx <= t) ? gv[e] * ex2(c2t - c2[sidx]) * dts[sidx] : 0.f;
-            }
-          }
-#pragma unroll
-          for (int cc = 0; cc < 8; ++cc)
-            st_shared_v4(wrow + ((cc ^ (tl & 7)) << 4), pack_bf16x2(gv[8 * cc + 0], gv[8 * cc + 1]),
-                         pack_bf16x2(gv[8 * cc + 2], gv[8 * cc + 3]), pack_bf16x2(gv[8 * cc + 4], gv[8 * cc + 5]),
-                         pack_bf16x2(gv[8 * cc + 6], gv[8 * cc + 7]));
+          for (int m = 0; m < 4; ++m)
+            o4[m] = pack_bf16x2(__uint_as_float(w4[m] << 16) * vv, __uint_as_float(w4[m] & 0xffff0000u) * vv);
+          st_shared_v4(addr, o4[0], o4[1], o4[2], o4[3]);
         }
       }
       fence_proxy_async_smem();
       tc_fence_before();
       named_barrier(1, 256);
-      if (tid == 0) mbar_arrive(&ms->w_full);
+      if (tid == 0 && ok) {
+        mbar_arrive(&ms->ops_ready[s]);
+        mbar_arrive(&ms->cum_free[cb]);
+      }
     }
-  } else {
+  } else if (warp < 14) {
     // ------------------------------------------------------------- output warps (128 threads)
     const int q = warp & 3;
     const int tl = q * 32 + lane;
@@ -558,15 +628,25 @@ k_chunk_scan_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
     for (int k = 0; k < nh; ++k) {
       const int s = k & 1, cb = k % K3_CUMBUF, h = h0 + k;
+      // x_t for the D x_t term, straight from global memory (the smem copy is scaled)
+      uint4 xg[8];
+      if (t < valid) {
+        const uint4 *xp = reinterpret_cast<const uint4 *>(x + (((size_t)bi * d.L + t0 + t) * d.H + h) * TP);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) xg[i] = __ldg(xp + i);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) xg[i] = make_uint4(0u, 0u, 0u, 0u);
+      }
       bool ok = mbar_wait(&ms->cum_full[cb], (k / K3_CUMBUF) & 1, abort_flag, err);
-      ok = ok && mbar_wait(&ms->x_full[s], (k >> 1) & 1, abort_flag, err);
       ok = ok && mbar_wait(&ms->acc_full[s], (k >> 1) & 1, abort_flag, err);
       tc_fence_after();
+      const uint32_t ys = smem_u32(base + K3Smem::x(s));  // the slot's x tile is consumed: stage y here
       if (ok) {
-        const float et = ex2(ms->c2[cb][t]);
+        const float c2t = ms->c2[cb][t];
+        const float et = ex2(c2t);
+        const float ut = ms->steep[cb] ? 1.f : ex2(c2t - ms->c2ref[cb]);
         const float Dh = D[h];
-        const uint32_t xrow = smem_u32(base + K3Smem::x(s)) + ti * 16384u + (uint32_t)tl * 128u;
-        float *yrow = y + (((size_t)bi * d.L + t0 + t) * d.H + h) * TP;
         const uint32_t acc = tmem + lane_off + TM_ACC + 128u * s;
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
@@ -574,33 +654,87 @@ k_chunk_scan_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
           tmem_ld32(acc + 32u * half, vi);
           tmem_ld32(acc + 64u + 32u * half, va);
           tmem_ld_wait();
-          if (t < valid) {
+          const uint32_t yrow = ys + half * 16384u + (uint32_t)tl * 128u;
 #pragma unroll
-            for (int cc = 0; cc < 4; ++cc) {
-              const int chunk = 4 * half + cc;
-              const uint4 xv = ld_shared_v4(xrow + ((chunk ^ (tl & 7)) << 4));
-              const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
-              float o[8];
+          for (int cc = 0; cc < 8; ++cc) {  // 8 chunks of 4 fp32 = the 32 channels of this half
+            const uint4 xw = xg[4 * half + cc / 2];
+            const uint32_t w0 = (cc & 1) ? xw.z : xw.x, w1 = (cc & 1) ? xw.w : xw.y;
+            const float xv[4] = {__uint_as_float(w0 << 16), __uint_as_float(w0 & 0xffff0000u),
+                                 __uint_as_float(w1 << 16), __uint_as_float(w1 & 0xffff0000u)};
+            float o[4];
 #pragma unroll
-              for (int m = 0; m < 4; ++m) {
-                const float xl = __uint_as_float(xw[m] << 16), xh = __uint_as_float(xw[m] & 0xffff0000u);
-                o[2 * m] = fmaf(et, vi[8 * cc + 2 * m], va[8 * cc + 2 * m]) + Dh * xl;
-                o[2 * m + 1] = fmaf(et, vi[8 * cc + 2 * m + 1], va[8 * cc + 2 * m + 1]) + Dh * xh;
-              }
-              float4 *dst = reinterpret_cast<float4 *>(yrow + 8 * chunk);
-              dst[0] = make_float4(o[0], o[1], o[2], o[3]);
-              dst[1] = make_float4(o[4], o[5], o[6], o[7]);
-            }
+            for (int m = 0; m < 4; ++m) o[m] = fmaf(et, vi[4 * cc + m], fmaf(ut, va[4 * cc + m], Dh * xv[m]));
+            st_shared_v4(yrow + ((cc ^ (tl & 7)) << 4), __float_as_uint(o[0]), __float_as_uint(o[1]),
+                         __float_as_uint(o[2]), __float_as_uint(o[3]));
           }
         }
       }
       tc_fence_before();
+      fence_proxy_async_smem();
       named_barrier(2, 128);
-      if (tid == 0) {
+      if (tid == 0 && ok) {
         mbar_arrive(&ms->acc_free[s]);
-        mbar_arrive(&ms->x_free[s]);
         mbar_arrive(&ms->cum_free[cb]);
+        tma_store_3d(&tm_y, base + K3Smem::x(s), h * TP, t0 + 128 * ti, bi);
+        tma_store_3d(&tm_y, base + K3Smem::x(s) + 16384u, h * TP + 32, t0 + 128 * ti, bi);
+        tma_store_commit();
+        tma_store_wait_read();
+        mbar_arrive(&ms->x_free[s]);
       }
+    }
+    if (tid == 0) tma_store_wait_all();
+  } else {
+    // ------------------------------------------------------------- decay-table warp
+    const int per = Q / 32;
+    for (int k = 0; k < nh; ++k) {
+      const int cb = k % K3_CUMBUF, h = h0 + k;
+      if (k >= K3_CUMBUF && !mbar_wait(&ms->cum_free[cb], ((k / K3_CUMBUF) - 1) & 1, abort_flag, err)) break;
+      const float a2 = A[h] * kLog2e;
+      float c2v[8], dtv[8];
+      float run = 0.f;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int tt = lane * per + j;
+        dtv[j] = (j < per && tt < valid) ? dt[((size_t)bi * d.L + t0 + tt) * d.H + h] : 0.f;
+        run += dtv[j] * a2;
+        c2v[j] = run;
+      }
+      float incl = run;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const float vv = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += vv;
+      }
+      const float excl = incl - run;
+      float *c2 = ms->c2[cb];
+      float *dts = ms->dts[cb];
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        if (j < per) {
+          c2[lane * per + j] = c2v[j] + excl;
+          dts[lane * per + j] = dtv[j];
+        }
+      __syncwarp();
+      const int ncol = 128 * nblk;
+      const int last = min(valid, ncol) - 1;
+      const float c2r = (ti > 0) ? c2[128 * ti - 1] : 0.f;
+      const float range = fabsf(c2r - c2[last]);
+      const int steep = !(range < kSteepLog2);  // also catches NaN
+      for (int sidx = lane; sidx < ncol; sidx += 32) ms->v[cb][sidx] = ex2(c2r - c2[sidx]) * dts[sidx];
+      if (steep) {
+        for (int sidx = lane; sidx < ncol; sidx += 32) {
+          const int g0 = sidx & ~31;
+          const float cs = c2[sidx], dv = dts[sidx];
+          ms->vo[cb][sidx] = ex2(c2[g0 + 31] - cs) * dv;
+          ms->vd[cb][sidx] = ex2(c2[g0] - cs) * dv;
+        }
+      }
+      if (lane == 0) {
+        ms->steep[cb] = steep;
+        ms->c2ref[cb] = c2r;
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ms->cum_full[cb]);
     }
   }
 
@@ -629,17 +763,22 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// 3-D bf16 tensor map {d0 (contiguous), d1, d2} with a {64, rows, 1} box and 128-byte swizzle.
-bool make_map(CUtensorMap *m, const void *ptr, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t rows) {
+// 3-D tensor map {d0 (contiguous), d1, d2}, box {inner, rows, 1}, 128-byte swizzle.
+bool make_map_t(CUtensorMap *m, CUtensorMapDataType type, uint32_t esize, const void *ptr, uint64_t d0, uint64_t d1,
+                uint64_t d2, uint32_t inner, uint32_t rows) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   const cuuint64_t dims[3] = {d0, d1, d2};
-  const cuuint64_t strides[2] = {d0 * 2, d0 * d1 * 2};
-  const cuuint32_t box[3] = {64, rows, 1};
+  const cuuint64_t strides[2] = {d0 * esize, d0 * d1 * esize};
+  const cuuint32_t box[3] = {inner, rows, 1};
   const cuuint32_t estr[3] = {1, 1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+  return fn(m, type, 3, const_cast<void *>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+// 3-D bf16 tensor map {d0 (contiguous), d1, d2} with a {64, rows, 1} box and 128-byte swizzle.
+bool make_map(CUtensorMap *m, const void *ptr, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t rows) {
+  return make_map_t(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ptr, d0, d1, d2, 64, rows);
 }
 
 int num_sms() {
@@ -651,21 +790,25 @@ int num_sms() {
   return n;
 }
 
-// Heads per CTA: the split of a group's heads that fills whole waves of CTAs best.
-int pick_heads_per_cta(int base_items, int hpg, int sms) {
-  int best_nhb = 1;
-  double best = -1.0;
+// Heads per CTA.  A CTA runs a fixed set-up (barriers, TMEM, the chunk's shared
+// operands: worth about `overhead` heads) and then its heads one after another; with one
+// CTA per SM, the kernel takes about waves x (heads per CTA + overhead).  Pick the split
+// of a group's heads that minimises that, preferring more CTAs on ties.
+int pick_heads_per_cta(int base_items, int hpg, int sms, double overhead) {
+  int best_kb = hpg;
+  double best = 1e30;
   for (int nhb = 1; nhb <= hpg; ++nhb) {
-    const long ctas = (long)base_items * nhb;
-    if (ctas > 4L * sms && nhb > 1) break;
+    const int kb = (hpg + nhb - 1) / nhb;
+    const int nblocks = (hpg + kb - 1) / kb;
+    const long ctas = (long)base_items * nblocks;
     const long waves = (ctas + sms - 1) / sms;
-    const double eff = (double)ctas / (double)(waves * sms);
-    if (eff > best + 1e-9) {
-      best = eff;
-      best_nhb = nhb;
+    const double cost = (double)waves * (kb + overhead);
+    if (cost <= best + 1e-9) {
+      best = cost;
+      best_kb = kb;
     }
   }
-  return (hpg + best_nhb - 1) / best_nhb;
+  return best_kb;
 }
 
 }  // namespace
@@ -679,12 +822,13 @@ cudaError_t launch_tc_prefill(const __nv_bfloat16 *x, const float *dt, const flo
                               const __nv_bfloat16 *C, const float *D, float *y, float *final_state, float *states,
                               float *cdecay, __nv_bfloat16 *hprev, int *err, const Dims &d, int Q, int nc,
                               cudaStream_t st, const cudaEvent_t *ev) {
-  CUtensorMap tm_x1, tm_B1, tm_x3, tm_C3, tm_B3, tm_h3;
+  CUtensorMap tm_x1, tm_B1, tm_x3, tm_C3, tm_B3, tm_h3, tm_y3;
   const uint64_t HP = (uint64_t)d.H * d.P, GN = (uint64_t)d.G * d.N;
   if (!make_map(&tm_x1, x, HP, d.L, d.b, Q) || !make_map(&tm_B1, B, GN, d.L, d.b, Q) ||
       !make_map(&tm_x3, x, HP, d.L, d.b, 128) || !make_map(&tm_C3, C, GN, d.L, d.b, 128) ||
       !make_map(&tm_B3, B, GN, d.L, d.b, 128) ||
-      !make_map(&tm_h3, hprev, (uint64_t)d.N, (uint64_t)d.P, (uint64_t)d.b * nc * d.H, 64))
+      !make_map(&tm_h3, hprev, (uint64_t)d.N, (uint64_t)d.P, (uint64_t)d.b * nc * d.H, 64) ||
+      !make_map_t(&tm_y3, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, y, HP, d.L, d.b, 32, 128))
     return cudaErrorInvalidValue;
   const int sms = num_sms();
   auto mark = [&](int i) { return ev ? cudaEventRecord(ev[i], st) : cudaSuccess; };
@@ -693,7 +837,7 @@ cudaError_t launch_tc_prefill(const __nv_bfloat16 *x, const float *dt, const flo
   // K1
   {
     const int base_items = d.b * nc * d.G;
-    const int kb = pick_heads_per_cta(base_items, d.hpg, sms);
+    const int kb = pick_heads_per_cta(base_items, d.hpg, sms, 1.0);
     const int nhb = (d.hpg + kb - 1) / kb;
     const size_t smem = tc_prefill_smem_k1(Q);
     e = cudaFuncSetAttribute(k_chunk_state_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -705,7 +849,7 @@ cudaError_t launch_tc_prefill(const __nv_bfloat16 *x, const float *dt, const flo
   if ((e = mark(1)) != cudaSuccess) return e;
   // K2
   {
-    const int per_head = d.P * d.N / 8;
+    const int per_head = d.P * d.N / 4;
     k_state_passing_bf16<<<dim3(d.b * d.H, (per_head + 255) / 256), 256, 0, st>>>(states, cdecay, hprev, final_state,
                                                                                  d, nc);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
@@ -715,12 +859,12 @@ cudaError_t launch_tc_prefill(const __nv_bfloat16 *x, const float *dt, const flo
   {
     const int ntt = Q / 128;
     const int base_items = d.b * nc * ntt * d.G;
-    const int kb = pick_heads_per_cta(base_items, d.hpg, sms);
+    const int kb = pick_heads_per_cta(base_items, d.hpg, sms, 2.0);
     const int nhb = (d.hpg + kb - 1) / kb;
     e = cudaFuncSetAttribute(k_chunk_scan_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kK3SmemBytes);
     if (e != cudaSuccess) return e;
     k_chunk_scan_tc<<<(unsigned)(base_items * nhb), K3_THREADS, kK3SmemBytes, st>>>(
-        tm_x3, tm_C3, tm_B3, tm_h3, dt, A, D, y, err, d, Q, nc, kb, nhb);
+        tm_x3, tm_C3, tm_B3, tm_h3, tm_y3, x, dt, A, D, err, d, Q, nc, kb, nhb);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   return mark(3);

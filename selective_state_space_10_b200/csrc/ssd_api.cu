@@ -5,7 +5,7 @@
 #include <stdint.h>
 #include <string.h>
 
-#include "../../include/ssd.h"
+#include "ssd.h"
 #include "kernels.h"
 
 namespace {
