@@ -7,7 +7,7 @@
 //
 //  K1 k_chunk_state_tc   S_c^T[n, p] = sum_t B_t[n] * (exp(cum_end - cum_t) dt_t x_t[p])
 //                        One CTA per (batch, chunk, group, block of heads).  TMA brings
-//                        B_c (once) and each head's x tile (ring of 2 slots); four warps
+//                        B_c (once) and each head's x tile (ring of 3 slots); eight warps
 //                        scale x's rows by the decay weight in fp32 and split the product
 //                        into a bf16 high part and a bf16 remainder; one thread issues
 //                        tcgen05.mma for both (M = 128 d_state rows, N = 64 channels,
@@ -51,21 +51,21 @@ constexpr int TP = 64;    // headdim handled by the tensor-core path
 constexpr int TN = 128;   // d_state handled by the tensor-core path
 
 // ============================================================================ K1
-constexpr int K1_SLOTS = 2;
+constexpr int K1_SLOTS = 3;
 constexpr int K1_CUMBUF = 3;
-constexpr int K1_THREADS = 352;  // warp 0 TMA, 1 MMA, 2-5 scale, 6-9 epilogue, 10 decay weights
+constexpr int K1_THREADS = 480;  // warp 0 TMA, 1 MMA, 2-9 scale, 10-13 epilogue, 14 decay weights
 
 struct K1Smem {
   // offsets from the 1024-aligned base
   static constexpr uint32_t bm = 0;  // B chunk: 2 x [Q][128 B]
-  // slot s: x (scaled in place to the bf16 high part) at x(), the bf16 remainder at lo()
-  __host__ __device__ static constexpr uint32_t x(int Q, int s) { return 2u * Q * 128u + (uint32_t)s * 2u * Q * 128u; }
-  __host__ __device__ static constexpr uint32_t lo(int Q, int s) { return x(Q, s) + (uint32_t)Q * 128u; }
-  __host__ __device__ static constexpr uint32_t misc(int Q) { return 2u * Q * 128u + K1_SLOTS * 2u * Q * 128u; }
+  // x slots (scaled in place to the bf16 high part), then one buffer for the bf16 remainder
+  __host__ __device__ static constexpr uint32_t x(int Q, int s) { return 2u * Q * 128u + (uint32_t)s * Q * 128u; }
+  __host__ __device__ static constexpr uint32_t lo(int Q) { return (2u + K1_SLOTS) * Q * 128u; }
+  __host__ __device__ static constexpr uint32_t misc(int Q) { return (3u + K1_SLOTS) * Q * 128u; }
 };
 
 struct K1Misc {
-  uint64_t b_full;
+  uint64_t b_full, lo_free;
   uint64_t x_full[K1_SLOTS], scaled[K1_SLOTS], x_free[K1_SLOTS];
   uint64_t acc_full[2], acc_free[2];
   uint64_t w_full[K1_CUMBUF], w_free[K1_CUMBUF];
@@ -98,6 +98,7 @@ k_chunk_state_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
 
   if (threadIdx.x == 0) {
     mbar_init(&ms->b_full, 1);
+    mbar_init(&ms->lo_free, 1);
     for (int s = 0; s < K1_SLOTS; ++s) {
       mbar_init(&ms->x_full[s], 1);
       mbar_init(&ms->scaled[s], 1);
@@ -159,7 +160,7 @@ k_chunk_state_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
         if (k >= 2 && !mbar_wait(&ms->acc_free[a], ((k >> 1) - 1) & 1, abort_flag, err)) break;
         tc_fence_after();
         const uint32_t x_addr = smem_u32(base + K1Smem::x(Q, s));
-        const uint32_t lo_addr = smem_u32(base + K1Smem::lo(Q, s));
+        const uint32_t lo_addr = smem_u32(base + K1Smem::lo(Q));
         for (int ks = 0; ks < Q / 16; ++ks) {
           // A = B chunk as [M = d_state][K = token], d_state contiguous (two 64-wide blocks Q*128 B apart)
           const uint64_t ad = smem_desc_sw128(bm_addr + ks * 2048u, (uint32_t)Q * 128u, 1024u);
@@ -171,21 +172,24 @@ k_chunk_state_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
         }
         mma_commit(&ms->acc_full[a]);
         mma_commit(&ms->x_free[s]);
+        mma_commit(&ms->lo_free);
       }
     }
     __syncwarp();
-  } else if (warp < 6) {
-    // ------------------------------------------------------------- scale warps (128 threads)
+  } else if (warp < 10) {
+    // ------------------------------------------------------------- scale warps (256 threads)
     const int tid = threadIdx.x - 64;
     for (int k = 0; k < nh; ++k) {
       const int s = k % K1_SLOTS, wb = k % K1_CUMBUF;
       bool ok = mbar_wait(&ms->w_full[wb], (k / K1_CUMBUF) & 1, abort_flag, err);
       ok = ok && mbar_wait(&ms->x_full[s], (k / K1_SLOTS) & 1, abort_flag, err);
+      if (k >= 1) ok = ok && mbar_wait(&ms->lo_free, (k - 1) & 1, abort_flag, err);  // previous MMA read lo
       if (ok) {
         const uint32_t xs = smem_u32(base + K1Smem::x(Q, s));
-        const uint32_t ls = smem_u32(base + K1Smem::lo(Q, s));
+        const uint32_t ls = smem_u32(base + K1Smem::lo(Q));
         const float *wv_row = ms->w[wb];
-        for (int unit = tid; unit < Q * 8; unit += 128) {
+#pragma unroll 4
+        for (int unit = tid; unit < Q * 8; unit += 256) {
           const float wv = wv_row[unit >> 3];
           const uint32_t off = (uint32_t)unit * 16u;  // rows are 128 B: unit*16 = row*128 + chunk*16
           const uint4 v = ld_shared_v4(xs + off);
@@ -204,17 +208,17 @@ k_chunk_state_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
         }
       }
       fence_proxy_async_smem();
-      named_barrier(1, 128);
+      named_barrier(1, 256);
       if (tid == 0 && ok) {
         mbar_arrive(&ms->scaled[s]);
         mbar_arrive(&ms->w_free[wb]);
       }
     }
-  } else if (warp < 10) {
+  } else if (warp < 14) {
     // ------------------------------------------------------------- epilogue warps (128 threads)
     const int q = warp & 3;
     const int n = q * 32 + lane;  // d_state row of the accumulator
-    const int tid = threadIdx.x - 192;
+    const int tid = threadIdx.x - 320;
     for (int k = 0; k < nh; ++k) {
       const int a = k & 1, h = h0 + k;
       const bool ok = mbar_wait(&ms->acc_full[a], (k >> 1) & 1, abort_flag, err);
@@ -343,7 +347,9 @@ struct K3Smem {
   // x tiles: nblk blocks of [128 rows][128 B]; after the head's MMAs, y staging (2 x [128][128 B])
   __host__ __device__ static constexpr uint32_t x(int s) { return 98304u + (uint32_t)s * 32768u; }  // 2 x 32 KB
   __host__ __device__ static constexpr uint32_t hs(int s) { return 163840u + (uint32_t)s * 16384u; } // 2 x 16 KB
-  static constexpr uint32_t misc = 196608u;
+  // y staging: one [32 rows][128 B] buffer per output warp (4 x 4 KB)
+  __host__ __device__ static constexpr uint32_t ystage(int w) { return 196608u + (uint32_t)w * 4096u; }
+  static constexpr uint32_t misc = 212992u;
 };
 
 struct K3Misc {
@@ -358,13 +364,8 @@ struct K3Misc {
   alignas(16) float c2[K3_CUMBUF][256];   // in-chunk cumulative log2-decay
   alignas(16) float dts[K3_CUMBUF][256];  // dt of each token of the chunk (0 past the end)
   alignas(16) float v[K3_CUMBUF][256];    // 2^(c2_r - c2_s) dt_s, s < 128 * (ti + 1)
-  // steep heads only (per-32-token references):
-  alignas(16) float vo[K3_CUMBUF][256];   // ref = last token of s's 32-token group
-  alignas(16) float vd[K3_CUMBUF][256];   // ref = first token of s's 32-token group
 };
-static_assert(offsetof(K3Misc, c2) % 16 == 0 && offsetof(K3Misc, v) % 16 == 0 && offsetof(K3Misc, vo) % 16 == 0 &&
-                  offsetof(K3Misc, vd) % 16 == 0,
-              "decay tables must be 16-byte aligned");
+static_assert(offsetof(K3Misc, c2) % 16 == 0 && offsetof(K3Misc, v) % 16 == 0, "decay tables must be 16-byte aligned");
 static_assert(K3Smem::misc % 16 == 0, "K3Misc must start 16-byte aligned");
 
 constexpr size_t kK3SmemBytes = 1024 + K3Smem::misc + sizeof(K3Misc);
@@ -381,8 +382,8 @@ __device__ __forceinline__ void st_row_bf16(uint32_t row_addr, int row, int cc0,
 __global__ void __launch_bounds__(K3_THREADS, 1)
 k_chunk_scan_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_C,
                 const __grid_constant__ CUtensorMap tm_B, const __grid_constant__ CUtensorMap tm_h,
-                const __grid_constant__ CUtensorMap tm_y, const __nv_bfloat16 *__restrict__ x,
-                const float *__restrict__ dt, const float *__restrict__ A, const float *__restrict__ D, int *err,
+                const __nv_bfloat16 *__restrict__ x, const float *__restrict__ dt, const float *__restrict__ A,
+                const float *__restrict__ D, float *__restrict__ y, int *err,
                 Dims d, int Q, int nc, int kb, int nhb) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -412,7 +413,7 @@ k_chunk_scan_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
     for (int s = 0; s < 2; ++s) {
       mbar_init(&ms->x_full[s], 1);
       mbar_init(&ms->ops_ready[s], 1);
-      mbar_init(&ms->x_free[s], 2);  // MMA commit + output (y staged out of the slot)
+      mbar_init(&ms->x_free[s], 1);  // MMA commit
       mbar_init(&ms->acc_full[s], 1);
       mbar_init(&ms->acc_free[s], 1);
     }
@@ -441,7 +442,6 @@ k_chunk_scan_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
       tma_prefetch_desc(&tm_C);
       tma_prefetch_desc(&tm_B);
       tma_prefetch_desc(&tm_h);
-      tma_prefetch_desc(&tm_y);
       mbar_arrive_expect_tx(&ms->cb_full, 32768u + (uint32_t)nblk * 32768u);
       for (int kn = 0; kn < 2; ++kn)
         tma_load_3d(base + K3Smem::cm + kn * 16384u, &tm_C, &ms->cb_full, g * TN + 64 * kn, t0 + 128 * ti, bi);
@@ -564,25 +564,13 @@ k_chunk_scan_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                 const float *vf = ms->v[cb] + col0;  // reference r: the column factors of x scaling
 #pragma unroll
                 for (int e = 0; e < 32; ++e) gg[e] *= vf[e] * u;
-              } else if (grp < q) {
-                const float u = ex2(c2t - c2[col0 + 31]);
-                const float *vo = ms->vo[cb] + col0;
+              } else {
+                // a steep head's own tile: one exp of a difference per element (never overflows)
+                const float *dts = ms->dts[cb];
 #pragma unroll
-                for (int e = 0; e < 32; ++e) gg[e] *= vo[e] * u;
-              } else {  // grp == q: own 32-token group, masked
-                const float range = c2[col0] - c2[col0 + 31];
-                if (fabsf(range) < kSteepLog2) {
-                  const float u = ex2(c2t - c2[col0]);
-                  const float *vd = ms->vd[cb] + col0;
-#pragma unroll
-                  for (int e = 0; e < 32; ++e) gg[e] = (col0 + e <= t) ? gg[e] * (vd[e] * u) : 0.f;
-                } else {  // decay too steep even inside the group: one exp per element
-                  const float *dts = ms->dts[cb];
-#pragma unroll
-                  for (int e = 0; e < 32; ++e) {
-                    const int sidx = col0 + e;
-                    gg[e] = (sidx <= t) ? gg[e] * ex2(c2t - c2[sidx]) * dts[sidx] : 0.f;
-                  }
+                for (int e = 0; e < 32; ++e) {
+                  const int sidx = col0 + e;
+                  gg[e] = (sidx <= t) ? gg[e] * ex2(c2t - c2[sidx]) * dts[sidx] : 0.f;
                 }
               }
             }
@@ -621,11 +609,15 @@ k_chunk_scan_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
     }
   } else if (warp < 14) {
     // ------------------------------------------------------------- output warps (128 threads)
+    // Each warp owns 32 rows (TMEM lane quarter q).  A 32-column half of its rows goes
+    // through the warp's own 4 KB swizzled staging buffer, then out with full-line stores
+    // (8 threads per 128-byte row segment).
     const int q = warp & 3;
     const int tl = q * 32 + lane;
     const int t = 128 * ti + tl;
     const int tid = threadIdx.x - 320;
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+    const uint32_t stg = smem_u32(base + K3Smem::ystage(warp - 10));
     for (int k = 0; k < nh; ++k) {
       const int s = k & 1, cb = k % K3_CUMBUF, h = h0 + k;
       // x_t for the D x_t term, straight from global memory (the smem copy is scaled)
@@ -641,20 +633,21 @@ k_chunk_scan_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
       bool ok = mbar_wait(&ms->cum_full[cb], (k / K3_CUMBUF) & 1, abort_flag, err);
       ok = ok && mbar_wait(&ms->acc_full[s], (k >> 1) & 1, abort_flag, err);
       tc_fence_after();
-      const uint32_t ys = smem_u32(base + K3Smem::x(s));  // the slot's x tile is consumed: stage y here
       if (ok) {
         const float c2t = ms->c2[cb][t];
         const float et = ex2(c2t);
         const float ut = ms->steep[cb] ? 1.f : ex2(c2t - ms->c2ref[cb]);
         const float Dh = D[h];
         const uint32_t acc = tmem + lane_off + TM_ACC + 128u * s;
+        const int rbase = t0 + 128 * ti + 32 * q;  // first (chunk-absolute) row of this warp
+        float *ybase = y + (((size_t)bi * d.L + rbase) * d.H + h) * TP;
+        const size_t yrow_stride = (size_t)d.H * TP;
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
           float vi[32], va[32];
           tmem_ld32(acc + 32u * half, vi);
           tmem_ld32(acc + 64u + 32u * half, va);
           tmem_ld_wait();
-          const uint32_t yrow = ys + half * 16384u + (uint32_t)tl * 128u;
 #pragma unroll
           for (int cc = 0; cc < 8; ++cc) {  // 8 chunks of 4 fp32 = the 32 channels of this half
             const uint4 xw = xg[4 * half + cc / 2];
@@ -664,25 +657,27 @@ k_chunk_scan_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
             float o[4];
 #pragma unroll
             for (int m = 0; m < 4; ++m) o[m] = fmaf(et, vi[4 * cc + m], fmaf(ut, va[4 * cc + m], Dh * xv[m]));
-            st_shared_v4(yrow + ((cc ^ (tl & 7)) << 4), __float_as_uint(o[0]), __float_as_uint(o[1]),
-                         __float_as_uint(o[2]), __float_as_uint(o[3]));
+            st_shared_v4(stg + (uint32_t)lane * 128u + ((cc ^ (lane & 7)) << 4), __float_as_uint(o[0]),
+                         __float_as_uint(o[1]), __float_as_uint(o[2]), __float_as_uint(o[3]));
           }
+          __syncwarp();
+#pragma unroll
+          for (int it = 0; it < 8; ++it) {  // rows 4*it .. 4*it+3 of the warp, 8 threads per row
+            const int rr = 4 * it + (lane >> 3), cc = lane & 7;
+            const uint4 v = ld_shared_v4(stg + (uint32_t)rr * 128u + ((cc ^ (rr & 7)) << 4));
+            if (128 * ti + 32 * q + rr < valid)
+              *reinterpret_cast<uint4 *>(ybase + (size_t)rr * yrow_stride + 32 * half + 4 * cc) = v;
+          }
+          __syncwarp();
         }
       }
       tc_fence_before();
-      fence_proxy_async_smem();
       named_barrier(2, 128);
       if (tid == 0 && ok) {
         mbar_arrive(&ms->acc_free[s]);
         mbar_arrive(&ms->cum_free[cb]);
-        tma_store_3d(&tm_y, base + K3Smem::x(s), h * TP, t0 + 128 * ti, bi);
-        tma_store_3d(&tm_y, base + K3Smem::x(s) + 16384u, h * TP + 32, t0 + 128 * ti, bi);
-        tma_store_commit();
-        tma_store_wait_read();
-        mbar_arrive(&ms->x_free[s]);
       }
     }
-    if (tid == 0) tma_store_wait_all();
   } else {
     // ------------------------------------------------------------- decay-table warp
     const int per = Q / 32;
@@ -721,14 +716,6 @@ k_chunk_scan_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
       const float range = fabsf(c2r - c2[last]);
       const int steep = !(range < kSteepLog2);  // also catches NaN
       for (int sidx = lane; sidx < ncol; sidx += 32) ms->v[cb][sidx] = ex2(c2r - c2[sidx]) * dts[sidx];
-      if (steep) {
-        for (int sidx = lane; sidx < ncol; sidx += 32) {
-          const int g0 = sidx & ~31;
-          const float cs = c2[sidx], dv = dts[sidx];
-          ms->vo[cb][sidx] = ex2(c2[g0 + 31] - cs) * dv;
-          ms->vd[cb][sidx] = ex2(c2[g0] - cs) * dv;
-        }
-      }
       if (lane == 0) {
         ms->steep[cb] = steep;
         ms->c2ref[cb] = c2r;
@@ -822,13 +809,12 @@ cudaError_t launch_tc_prefill(const __nv_bfloat16 *x, const float *dt, const flo
                               const __nv_bfloat16 *C, const float *D, float *y, float *final_state, float *states,
                               float *cdecay, __nv_bfloat16 *hprev, int *err, const Dims &d, int Q, int nc,
                               cudaStream_t st, const cudaEvent_t *ev) {
-  CUtensorMap tm_x1, tm_B1, tm_x3, tm_C3, tm_B3, tm_h3, tm_y3;
+  CUtensorMap tm_x1, tm_B1, tm_x3, tm_C3, tm_B3, tm_h3;
   const uint64_t HP = (uint64_t)d.H * d.P, GN = (uint64_t)d.G * d.N;
   if (!make_map(&tm_x1, x, HP, d.L, d.b, Q) || !make_map(&tm_B1, B, GN, d.L, d.b, Q) ||
       !make_map(&tm_x3, x, HP, d.L, d.b, 128) || !make_map(&tm_C3, C, GN, d.L, d.b, 128) ||
       !make_map(&tm_B3, B, GN, d.L, d.b, 128) ||
-      !make_map(&tm_h3, hprev, (uint64_t)d.N, (uint64_t)d.P, (uint64_t)d.b * nc * d.H, 64) ||
-      !make_map_t(&tm_y3, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, y, HP, d.L, d.b, 32, 128))
+      !make_map(&tm_h3, hprev, (uint64_t)d.N, (uint64_t)d.P, (uint64_t)d.b * nc * d.H, 64))
     return cudaErrorInvalidValue;
   const int sms = num_sms();
   auto mark = [&](int i) { return ev ? cudaEventRecord(ev[i], st) : cudaSuccess; };
@@ -864,7 +850,7 @@ cudaError_t launch_tc_prefill(const __nv_bfloat16 *x, const float *dt, const flo
     e = cudaFuncSetAttribute(k_chunk_scan_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kK3SmemBytes);
     if (e != cudaSuccess) return e;
     k_chunk_scan_tc<<<(unsigned)(base_items * nhb), K3_THREADS, kK3SmemBytes, st>>>(
-        tm_x3, tm_C3, tm_B3, tm_h3, tm_y3, x, dt, A, D, err, d, Q, nc, kb, nhb);
+        tm_x3, tm_C3, tm_B3, tm_h3, x, dt, A, D, y, err, d, Q, nc, kb, nhb);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   return mark(3);
