@@ -161,6 +161,34 @@ SSD_API const char *ssd_prefill_kernel_name(const ssd_dims *dims, ssd_dtype dtyp
 SSD_API ssd_status ssd_prefill_device_status(const void *workspace, size_t workspace_bytes, ssd_stream_t stream);
 
 /*
+ * ssd_prefill for callers that cannot allocate device memory.  Some callers cannot call
+ * cudaMalloc or provide device memory of their own: plugins inside a host process whose
+ * device allocator belongs to the host framework, and serving loops that forbid any
+ * allocation once running.  This call takes no workspace: its scratch is a fixed array
+ * of ssd_prefill_noalloc_max_workspace() bytes (32 MiB) compiled into the library.  It
+ * computes exactly what ssd_prefill computes, with the same arguments otherwise.
+ * (The pages describe no such call; it serves these callers only.)
+ *
+ *   - Allocates nothing: no cudaMalloc, cudaFree or allocating library routine.  The
+ *     array is held on a device, until the process exits, from the first call on it.
+ *   - The first call on a device, with that device current, looks up the array's device
+ *     address (cudaGetSymbolAddress) and caches it; make that first call before any
+ *     stream capture.
+ *   - Every call shares the one array: calls whose executions overlap on the GPU (other
+ *     streams, other host threads without ordering) race and give undefined results.
+ *     Order them on one stream or synchronise between them.
+ *   - Errors: as ssd_prefill; SSD_ERR_WORKSPACE if ssd_prefill_workspace_size() for these
+ *     arguments exceeds the array (the 2.7B-shaped 4096-token layer needs more; the
+ *     130M-shaped one fits).  SSD_ERR_CUDA if the address look-up fails.
+ */
+SSD_API ssd_status ssd_prefill_noalloc(const ssd_dims *dims, ssd_dtype dtype, const void *x, const float *dt,
+                                       const float *A, const void *B, const void *C, const float *D, int chunk,
+                                       float *y, float *final_state, ssd_stream_t stream);
+
+/* Size in bytes of the fixed scratch array ssd_prefill_noalloc uses (32 MiB). */
+SSD_API size_t ssd_prefill_noalloc_max_workspace(void);
+
+/*
  * One cached decode step (O(1) in the sequence length: "Compiler-First State Space
  * Duality ..." abstract; the recurrent mode of "Mamba and Selective State Space Models"
  * section 3).  Reads state = h_{t-1}, overwrites it in place with h_t, writes y_t.

@@ -259,3 +259,17 @@ ssd_status ssd_decode_step(const ssd_dims *dims, ssd_dtype dtype, float *state, 
 }
 
 }  // extern "C"
+
+namespace ssd {
+
+// Internal entry for other translation units of the library: ssd_prefill with a given
+// workspace (same validation, computation and errors).
+ssd_status prefill_into_workspace(const ssd_dims *dims, ssd_dtype dtype, const void *x, const float *dt,
+                                  const float *A, const void *B, const void *C, const float *D, int chunk,
+                                  float *y, float *final_state, void *workspace, size_t workspace_bytes,
+                                  ssd_stream_t stream) {
+  return prefill_impl(dims, dtype, x, dt, A, B, C, D, chunk, y, final_state, workspace, workspace_bytes, stream,
+                      nullptr, 0, false);
+}
+
+}  // namespace ssd

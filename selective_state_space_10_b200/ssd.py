@@ -33,7 +33,8 @@ class Dims(ctypes.Structure):
 # Every symbol include/ssd.h declares.
 EXPORTS = ("ssd_status_string", "ssd_version", "ssd_prefill_workspace_size",
            "ssd_prefill_kernel_launches", "ssd_prefill", "ssd_prefill_timed",
-           "ssd_prefill_kernel_name", "ssd_prefill_device_status", "ssd_decode_step")
+           "ssd_prefill_kernel_name", "ssd_prefill_device_status", "ssd_prefill_noalloc",
+           "ssd_prefill_noalloc_max_workspace", "ssd_decode_step")
 
 
 def _load():
@@ -60,6 +61,10 @@ def _load():
     lib.ssd_prefill_kernel_name.restype = ctypes.c_char_p
     lib.ssd_prefill_device_status.argtypes = [vp, sz, vp]
     lib.ssd_prefill_device_status.restype = ci
+    lib.ssd_prefill_noalloc.argtypes = [dp, ci, vp, fp, fp, vp, vp, fp, ci, fp, fp, vp]
+    lib.ssd_prefill_noalloc.restype = ci
+    lib.ssd_prefill_noalloc_max_workspace.argtypes = []
+    lib.ssd_prefill_noalloc_max_workspace.restype = sz
     lib.ssd_decode_step.argtypes = [dp, ci, fp, vp, fp, fp, vp, vp, fp, fp, vp]
     lib.ssd_decode_step.restype = ci
     return lib
@@ -166,6 +171,40 @@ def prefill(x, dt, A, B, C, D, chunk: int = 256, y=None, final_state=None, works
     if st != OK:
         raise SSDError(st, "ssd_prefill")
     return y, final_state
+
+
+def prefill_noalloc(x, dt, A, B, C, D, chunk: int = 256, y=None, final_state=None,
+                    stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """ssd_prefill_noalloc: the same prefill, with no workspace argument.  For callers
+    that cannot allocate device memory, the library takes its scratch from a fixed array
+    of prefill_noalloc_max_workspace() bytes; calls that overlap on the GPU race on it.
+    (Outputs are still allocated here when not given; pass y and final_state to avoid
+    that.)"""
+    b, L, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    dev = x.device
+    for name, t, shape, dtype in (("dt", dt, (b, L, H), torch.float32), ("A", A, (H,), torch.float32),
+                                  ("B", B, (b, L, G, N), x.dtype), ("C", C, (b, L, G, N), x.dtype),
+                                  ("D", D, (H,), torch.float32)):
+        _check(t, name, shape, dtype, dev)
+    if x.dtype not in _DTYPES:
+        raise ValueError(f"unsupported input dtype {x.dtype}")
+    if y is None:
+        y = torch.empty((b, L, H, P), dtype=torch.float32, device=dev)
+    if final_state is None:
+        final_state = torch.empty((b, H, P, N), dtype=torch.float32, device=dev)
+    _check(y, "y", (b, L, H, P), torch.float32, dev)
+    _check(final_state, "final_state", (b, H, P, N), torch.float32, dev)
+    st = lib.ssd_prefill_noalloc(ctypes.byref(dims_of_prefill(x, B)), _DTYPES[x.dtype], _ptr(x), _ptr(dt),
+                                 _ptr(A), _ptr(B), _ptr(C), _ptr(D), int(chunk), _ptr(y), _ptr(final_state),
+                                 _stream(stream))
+    if st != OK:
+        raise SSDError(st, "ssd_prefill_noalloc")
+    return y, final_state
+
+
+def prefill_noalloc_max_workspace() -> int:
+    return lib.ssd_prefill_noalloc_max_workspace()
 
 
 def prefill_device_status(workspace, stream=None) -> int:

@@ -148,3 +148,15 @@ def test_empty_batch_is_a_no_op(ssd):
     assert _prefill(ssd, d, ptrs=null, ws=0, ws_bytes=0) == ssd.OK
     nd = {k: None for k in ("state", "x", "dt", "A", "B", "C", "D", "y")}
     assert _decode(ssd, d, ptrs=nd) == ssd.OK
+
+
+def test_noalloc_validation_without_a_gpu(ssd):
+    """ssd_prefill_noalloc rejects invalid and oversized problems before any CUDA call."""
+    f = ssd.lib.ssd_prefill_noalloc
+    v = ctypes.c_void_p(FAKE)
+    assert ssd.prefill_noalloc_max_workspace() == 32 << 20
+    assert f(None, 1, v, v, v, v, v, v, 256, v, v, None) == ssd.ERR_INVALID_ARG
+    big = _dims(ssd, b=1, L=4096, H=80)
+    assert ssd.prefill_workspace_size(big, 1, 256) > ssd.prefill_noalloc_max_workspace()
+    assert f(ctypes.byref(big), 1, v, v, v, v, v, v, 256, v, v, None) == ssd.ERR_WORKSPACE
+    assert f(ctypes.byref(_dims(ssd)), 1, v, v, v, v, v, v, 48, v, v, None) == ssd.ERR_INVALID_ARG
