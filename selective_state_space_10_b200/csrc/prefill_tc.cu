@@ -7,24 +7,27 @@
 //
 //  K1 k_chunk_state_tc   S_c^T[n, p] = sum_t B_t[n] * (exp(cum_end - cum_t) dt_t x_t[p])
 //                        One CTA per (batch, chunk, group, block of heads).  TMA brings
-//                        B_c (once) and each head's x tile (ring of 3 slots); eight warps
+//                        B_c (once) and each head's x tile (ring of 2 slots); eight warps
 //                        scale x's rows by the decay weight in fp32 and split the product
-//                        into a bf16 high part and a bf16 remainder; one thread issues
-//                        tcgen05.mma for both (M = 128 d_state rows, N = 64 channels,
-//                        K = Q tokens, accumulated in TMEM), so the state is accurate to
-//                        fp32 level rather than bf16 level; four warps stream S_c out in
-//                        fp32.  Also writes the chunk's total decay exp(cum_end).
+//                        into a bf16 high part and a bf16 remainder, stored side by side;
+//                        one thread issues tcgen05.mma with both as the two 64-wide halves
+//                        of N = 128 (M = 128 d_state rows, K = Q tokens), and four warps
+//                        add the halves and stream S_c out in fp32, so the state is
+//                        accurate to fp32 level rather than bf16 level.  Also writes the
+//                        chunk's total decay exp(cum_end).
 //  K2 k_state_passing_bf16
 //                        h_c = exp(cum_end,c) h_{c-1} + S_c over chunks in fp32 (the
 //                        first-order recurrence of "Mamba and Selective State Space
 //                        Models" section 5); writes the state entering each chunk in bf16
 //                        (the next kernel's MMA operand) and the final state in fp32.
 //  K3 k_chunk_scan_tc    One CTA per (batch, chunk, 128-row token tile, group, block of
-//                        heads).  G = C_tile B_chunk^T is computed once into TMEM.  Per
-//                        head: 8 warps turn G into W = G o decay o dt (bf16, causal mask)
-//                        in shared memory; tcgen05.mma forms ACC_inter = C_tile h_prev^T
-//                        and ACC_intra = W X (double-buffered in TMEM across heads); four
-//                        warps write y_t = exp(cum_t) ACC_inter + ACC_intra + D x_t (fp32).
+//                        heads).  G = C_tile B_chunk^T is computed once into TMEM and,
+//                        masked, converted once to a head-independent bf16 W (see the
+//                        decay factorisation at K3 below); per head, 4 warps scale the
+//                        rows of its x tile by the column decay factors, tcgen05.mma forms
+//                        ACC_inter = C_tile h_prev^T and ACC_intra = W X' (double-buffered
+//                        in TMEM across heads), and 8 warps write
+//                        y_t = exp(cum_t) ACC_inter + u_t ACC_intra + D x_t (fp32).
 //
 // Numerics: every decay exp(cum_t - cum_s), s <= t, is formed so that no intermediate
 // leaves the range of the result: inside a 128-token block directly from the
@@ -51,21 +54,21 @@ constexpr int TP = 64;    // headdim handled by the tensor-core path
 constexpr int TN = 128;   // d_state handled by the tensor-core path
 
 // ============================================================================ K1
-constexpr int K1_SLOTS = 3;
+constexpr int K1_SLOTS = 2;
 constexpr int K1_CUMBUF = 3;
 constexpr int K1_THREADS = 480;  // warp 0 TMA, 1 MMA, 2-9 scale, 10-13 epilogue, 14 decay weights
 
 struct K1Smem {
   // offsets from the 1024-aligned base
   static constexpr uint32_t bm = 0;  // B chunk: 2 x [Q][128 B]
-  // x slots (scaled in place to the bf16 high part), then one buffer for the bf16 remainder
-  __host__ __device__ static constexpr uint32_t x(int Q, int s) { return 2u * Q * 128u + (uint32_t)s * Q * 128u; }
-  __host__ __device__ static constexpr uint32_t lo(int Q) { return (2u + K1_SLOTS) * Q * 128u; }
-  __host__ __device__ static constexpr uint32_t misc(int Q) { return (3u + K1_SLOTS) * Q * 128u; }
+  // slot s: x (scaled in place to the bf16 high part), directly followed by its remainder
+  __host__ __device__ static constexpr uint32_t x(int Q, int s) { return 2u * Q * 128u + (uint32_t)s * 2u * Q * 128u; }
+  __host__ __device__ static constexpr uint32_t lo(int Q, int s) { return x(Q, s) + (uint32_t)Q * 128u; }
+  __host__ __device__ static constexpr uint32_t misc(int Q) { return 2u * Q * 128u + K1_SLOTS * 2u * Q * 128u; }
 };
 
 struct K1Misc {
-  uint64_t b_full, lo_free;
+  uint64_t b_full;
   uint64_t x_full[K1_SLOTS], scaled[K1_SLOTS], x_free[K1_SLOTS];
   uint64_t acc_full[2], acc_free[2];
   uint64_t w_full[K1_CUMBUF], w_free[K1_CUMBUF];
@@ -98,7 +101,6 @@ k_chunk_state_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
 
   if (threadIdx.x == 0) {
     mbar_init(&ms->b_full, 1);
-    mbar_init(&ms->lo_free, 1);
     for (int s = 0; s < K1_SLOTS; ++s) {
       mbar_init(&ms->x_full[s], 1);
       mbar_init(&ms->scaled[s], 1);
@@ -116,7 +118,7 @@ k_chunk_state_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
     mbar_fence_init();
   }
   if (warp == 1) {
-    tmem_alloc(&ms->tmem, 128);
+    tmem_alloc(&ms->tmem, 256);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -151,7 +153,7 @@ k_chunk_state_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
   } else if (warp == 1) {
     // ------------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      const uint32_t idesc = idesc_bf16_f32(128, TP, /*a MN-major*/ true, /*b MN-major*/ true);
+      const uint32_t idesc = idesc_bf16_f32(128, 2 * TP, /*a MN-major*/ true, /*b MN-major*/ true);
       const uint32_t bm_addr = smem_u32(base + K1Smem::bm);
       bool ok = mbar_wait(&ms->b_full, 0, abort_flag, err);
       for (int k = 0; ok && k < nh; ++k) {
@@ -160,19 +162,15 @@ k_chunk_state_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
         if (k >= 2 && !mbar_wait(&ms->acc_free[a], ((k >> 1) - 1) & 1, abort_flag, err)) break;
         tc_fence_after();
         const uint32_t x_addr = smem_u32(base + K1Smem::x(Q, s));
-        const uint32_t lo_addr = smem_u32(base + K1Smem::lo(Q));
         for (int ks = 0; ks < Q / 16; ++ks) {
           // A = B chunk as [M = d_state][K = token], d_state contiguous (two 64-wide blocks Q*128 B apart)
           const uint64_t ad = smem_desc_sw128(bm_addr + ks * 2048u, (uint32_t)Q * 128u, 1024u);
-          // B = scaled x as [K = token][N = channel], channel contiguous: high part, then remainder
-          const uint64_t bh = smem_desc_sw128(x_addr + ks * 2048u, (uint32_t)Q * 128u, 1024u);
-          const uint64_t bl = smem_desc_sw128(lo_addr + ks * 2048u, (uint32_t)Q * 128u, 1024u);
-          mma_bf16(tmem + (uint32_t)(a * TP), ad, bh, idesc, ks > 0 ? 1u : 0u);
-          mma_bf16(tmem + (uint32_t)(a * TP), ad, bl, idesc, 1u);
+          // B = [K = token][N = (high | remainder) x channel]: two 64-wide blocks Q*128 B apart
+          const uint64_t bd = smem_desc_sw128(x_addr + ks * 2048u, (uint32_t)Q * 128u, 1024u);
+          mma_bf16(tmem + (uint32_t)(a * 2 * TP), ad, bd, idesc, ks > 0 ? 1u : 0u);
         }
         mma_commit(&ms->acc_full[a]);
         mma_commit(&ms->x_free[s]);
-        mma_commit(&ms->lo_free);
       }
     }
     __syncwarp();
@@ -183,10 +181,9 @@ k_chunk_state_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
       const int s = k % K1_SLOTS, wb = k % K1_CUMBUF;
       bool ok = mbar_wait(&ms->w_full[wb], (k / K1_CUMBUF) & 1, abort_flag, err);
       ok = ok && mbar_wait(&ms->x_full[s], (k / K1_SLOTS) & 1, abort_flag, err);
-      if (k >= 1) ok = ok && mbar_wait(&ms->lo_free, (k - 1) & 1, abort_flag, err);  // previous MMA read lo
       if (ok) {
         const uint32_t xs = smem_u32(base + K1Smem::x(Q, s));
-        const uint32_t ls = smem_u32(base + K1Smem::lo(Q));
+        const uint32_t ls = smem_u32(base + K1Smem::lo(Q, s));
         const float *wv_row = ms->w[wb];
 #pragma unroll 4
         for (int unit = tid; unit < Q * 8; unit += 256) {
@@ -227,11 +224,12 @@ k_chunk_state_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
         float *out = states + (((size_t)bi * nc + c) * d.H + h) * (size_t)(TP * TN) + n;
 #pragma unroll
         for (int cg = 0; cg < 2; ++cg) {
-          float v[32];
-          tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(a * TP + cg * 32), v);
+          float vh[32], vl[32];
+          tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(a * 2 * TP + cg * 32), vh);
+          tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(a * 2 * TP + TP + cg * 32), vl);
           tmem_ld_wait();
 #pragma unroll
-          for (int j = 0; j < 32; ++j) out[(size_t)(cg * 32 + j) * TN] = v[j];
+          for (int j = 0; j < 32; ++j) out[(size_t)(cg * 32 + j) * TN] = vh[j] + vl[j];
         }
       }
       tc_fence_before();
@@ -277,7 +275,7 @@ k_chunk_state_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 128);
+    tmem_dealloc(tmem, 256);
   }
 }
 
@@ -337,7 +335,7 @@ k_state_passing_bf16(const float *__restrict__ states, const float *__restrict__
 // every factor lies in [2^-100, 2^100] and all intermediates stay normal fp32).  Heads
 // with a steeper tile ("steep" heads) build their own W with per-32-token references
 // instead, as a slower exact fallback.
-constexpr int K3_THREADS = 480;  // warp 0 TMA, 1 MMA, 2-9 W/x scaling, 10-13 output, 14 decay tables
+constexpr int K3_THREADS = 480;  // warp 0 TMA, 1 MMA, 2-5 W/x scaling, 6-13 output, 14 decay tables
 constexpr int K3_CUMBUF = 3;
 constexpr float kSteepLog2 = 100.f;
 
@@ -347,8 +345,8 @@ struct K3Smem {
   // x tiles: nblk blocks of [128 rows][128 B]; after the head's MMAs, y staging (2 x [128][128 B])
   __host__ __device__ static constexpr uint32_t x(int s) { return 98304u + (uint32_t)s * 32768u; }  // 2 x 32 KB
   __host__ __device__ static constexpr uint32_t hs(int s) { return 163840u + (uint32_t)s * 16384u; } // 2 x 16 KB
-  // y staging: one [32 rows][128 B] buffer per output warp (4 x 4 KB)
-  __host__ __device__ static constexpr uint32_t ystage(int w) { return 196608u + (uint32_t)w * 4096u; }
+  // x/y staging: one [32 rows][64 B] buffer per output warp (8 x 2 KB)
+  __host__ __device__ static constexpr uint32_t ystage(int w) { return 196608u + (uint32_t)w * 2048u; }
   static constexpr uint32_t misc = 212992u;
 };
 
@@ -509,11 +507,11 @@ k_chunk_scan_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
       }
     }
     __syncwarp();
-  } else if (warp < 10) {
-    // ------------------------------------------------------------- W build and x scaling (256 threads)
-    // W builds: thread (q, ch, lane) owns row tl = 32q + lane, columns [64ch, 64ch + 64) of
-    // each source block (the warp's rows are the 32-token group q of the tile).
-    const int q = warp & 3, ch = (warp - 2) >> 2;
+  } else if (warp < 6) {
+    // ------------------------------------------------------------- W build and x scaling (128 threads)
+    // W builds: thread (q, lane) owns row tl = 32q + lane of every source block, in four
+    // 32-column groups (the warp's rows are the 32-token group q of the tile).
+    const int q = warp & 3;
     const int tl = q * 32 + lane;
     const int tid = threadIdx.x - 64;
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
@@ -533,49 +531,42 @@ k_chunk_scan_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
           const float *c2 = ms->c2[cb];
           const float c2t = c2[t];
           for (int j = 0; j < nblk; ++j) {
-            const uint32_t wrow = smem_u32(base + K3Smem::bw) + j * 32768u + ch * 16384u + (uint32_t)tl * 128u;
-            const int grp0 = 2 * ch;  // first of my two 32-column groups within block j
-            if (j == ti && grp0 > q) {  // both groups strictly right of the diagonal
-#pragma unroll
-              for (int cc = 0; cc < 8; ++cc) st_shared_v4(wrow + ((cc ^ (tl & 7)) << 4), 0u, 0u, 0u, 0u);
-              continue;
-            }
-            float gv[64];
-            tmem_ld32(tmem + lane_off + TM_G + (uint32_t)(128 * j + 64 * ch), *reinterpret_cast<float(*)[32]>(&gv[0]));
-            tmem_ld32(tmem + lane_off + TM_G + (uint32_t)(128 * j + 64 * ch + 32),
-                      *reinterpret_cast<float(*)[32]>(&gv[32]));
-            tmem_ld_wait();
-#pragma unroll
-            for (int gs = 0; gs < 2; ++gs) {
-              const int grp = grp0 + gs;
-              const int col0 = 128 * j + 32 * grp;  // chunk-relative first column
-              float *gg = &gv[32 * gs];
-              if (j == ti && grp > q) {
+            for (int grp = 0; grp < 4; ++grp) {
+              // 32 columns = 64 bytes = chunks 4*(grp&1) .. +3 of K-atom grp>>1
+              const uint32_t wrow =
+                  smem_u32(base + K3Smem::bw) + j * 32768u + (uint32_t)(grp >> 1) * 16384u + (uint32_t)tl * 128u;
+              const int cc0 = 4 * (grp & 1);
+              float gg[32];
+              if (j == ti && grp > q) {  // strictly right of the diagonal
 #pragma unroll
                 for (int e = 0; e < 32; ++e) gg[e] = 0.f;
-              } else if (!steep) {
-                // W_base = G o causal mask
-                if (j == ti && grp == q) {
-#pragma unroll
-                  for (int e = 0; e < 32; ++e) gg[e] = (col0 + e <= t) ? gg[e] : 0.f;
-                }
-              } else if (j < ti) {
-                const float u = ex2(c2t - c2[r]);
-                const float *vf = ms->v[cb] + col0;  // reference r: the column factors of x scaling
-#pragma unroll
-                for (int e = 0; e < 32; ++e) gg[e] *= vf[e] * u;
               } else {
-                // a steep head's own tile: one exp of a difference per element (never overflows)
-                const float *dts = ms->dts[cb];
+                const int col0 = 128 * j + 32 * grp;  // chunk-relative first column
+                tmem_ld32(tmem + lane_off + TM_G + (uint32_t)col0, gg);
+                tmem_ld_wait();
+                if (!steep) {
+                  // W_base = G o causal mask
+                  if (j == ti && grp == q) {
 #pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                  const int sidx = col0 + e;
-                  gg[e] = (sidx <= t) ? gg[e] * ex2(c2t - c2[sidx]) * dts[sidx] : 0.f;
+                    for (int e = 0; e < 32; ++e) gg[e] = (col0 + e <= t) ? gg[e] : 0.f;
+                  }
+                } else if (j < ti) {
+                  const float u = ex2(c2t - c2[r]);
+                  const float *vf = ms->v[cb] + col0;  // reference r: the column factors of x scaling
+#pragma unroll
+                  for (int e = 0; e < 32; ++e) gg[e] *= vf[e] * u;
+                } else {
+                  // a steep head's own tile: one exp of a difference per element (never overflows)
+                  const float *dts = ms->dts[cb];
+#pragma unroll
+                  for (int e = 0; e < 32; ++e) {
+                    const int sidx = col0 + e;
+                    gg[e] = (sidx <= t) ? gg[e] * ex2(c2t - c2[sidx]) * dts[sidx] : 0.f;
+                  }
                 }
               }
+              st_row_bf16(wrow, tl, cc0, gg);
             }
-            st_row_bf16(wrow, tl, 0, &gv[0]);
-            st_row_bf16(wrow, tl, 4, &gv[32]);
           }
           w_is_base = !steep;
         }
@@ -587,7 +578,7 @@ k_chunk_scan_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
         const float *vt = ms->v[cb];
         const int units = nblk * 128 * 8;  // 16-byte units: row = unit / 8 (rows of 128 B)
 #pragma unroll 4
-        for (int unit = tid; unit < units; unit += 256) {
+        for (int unit = tid; unit < units; unit += 128) {
           const float vv = vt[unit >> 3];
           const uint32_t addr = xs + (uint32_t)unit * 16u;
           const uint4 in = ld_shared_v4(addr);
@@ -601,78 +592,97 @@ k_chunk_scan_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
       }
       fence_proxy_async_smem();
       tc_fence_before();
-      named_barrier(1, 256);
+      named_barrier(1, 128);
       if (tid == 0 && ok) {
         mbar_arrive(&ms->ops_ready[s]);
         mbar_arrive(&ms->cum_free[cb]);
       }
     }
   } else if (warp < 14) {
-    // ------------------------------------------------------------- output warps (128 threads)
-    // Each warp owns 32 rows (TMEM lane quarter q).  A 32-column half of its rows goes
-    // through the warp's own 4 KB swizzled staging buffer, then out with full-line stores
-    // (8 threads per 128-byte row segment).
-    const int q = warp & 3;
+    // ------------------------------------------------------------- output warps (256 threads)
+    // Warp (q, hf) owns rows 32q .. 32q + 31 of the tile (TMEM lane quarter q) and the 32
+    // channels [32 hf, 32 hf + 32).  Its 2 KB staging buffer first brings in x (coalesced
+    // row segments) for the D x_t term, then takes y out 16 channels at a time, so every
+    // global access moves whole 64-byte row segments.
+    const int q = warp & 3, hf = (warp - 6) >> 2;
     const int tl = q * 32 + lane;
     const int t = 128 * ti + tl;
-    const int tid = threadIdx.x - 320;
+    const int tid = threadIdx.x - 192;
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
-    const uint32_t stg = smem_u32(base + K3Smem::ystage(warp - 10));
+    const uint32_t stg = smem_u32(base + K3Smem::ystage(warp - 6));
+    const int row0 = 128 * ti + 32 * q;                  // chunk-relative first row of the warp
+    const int nrows = max(0, min(32, valid - row0));     // rows of this warp that exist
+    // staging layout: 32 rows x 64 bytes, 16-byte chunk c of row r at (c ^ ((r >> 1) & 3))
+    auto sidx = [](int rr, int c) -> uint32_t { return (uint32_t)rr * 64u + ((c ^ ((rr >> 1) & 3)) << 4); };
     for (int k = 0; k < nh; ++k) {
       const int s = k & 1, cb = k % K3_CUMBUF, h = h0 + k;
-      // x_t for the D x_t term, straight from global memory (the smem copy is scaled)
-      uint4 xg[8];
-      if (t < valid) {
-        const uint4 *xp = reinterpret_cast<const uint4 *>(x + (((size_t)bi * d.L + t0 + t) * d.H + h) * TP);
+      // x rows of this warp (channels of its half), 4 threads per 64-byte row segment
+      const size_t rstride = (size_t)d.H * TP;  // elements between consecutive tokens
+      const __nv_bfloat16 *xw = x + (((size_t)bi * d.L + t0 + row0) * d.H + h) * TP + 32 * hf;
+      uint4 xl[4];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) xg[i] = __ldg(xp + i);
-      } else {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) xg[i] = make_uint4(0u, 0u, 0u, 0u);
+      for (int it = 0; it < 4; ++it) {
+        const int rr = 8 * it + (lane >> 2), c = lane & 3;
+        xl[it] = (rr < nrows) ? __ldg(reinterpret_cast<const uint4 *>(xw + (size_t)rr * rstride) + c)
+                              : make_uint4(0u, 0u, 0u, 0u);
       }
       bool ok = mbar_wait(&ms->cum_full[cb], (k / K3_CUMBUF) & 1, abort_flag, err);
       ok = ok && mbar_wait(&ms->acc_full[s], (k >> 1) & 1, abort_flag, err);
       tc_fence_after();
       if (ok) {
+        const uint32_t acc = tmem + lane_off + TM_ACC + 128u * s + 32u * hf;
+        float vi[32], va[32];
+        tmem_ld32(acc, vi);
+        tmem_ld32(acc + 64u, va);
+#pragma unroll
+        for (int it = 0; it < 4; ++it) {
+          const int rr = 8 * it + (lane >> 2), c = lane & 3;
+          st_shared_v4(stg + sidx(rr, c), xl[it].x, xl[it].y, xl[it].z, xl[it].w);
+        }
+        __syncwarp();
+        uint32_t xr[16];  // this thread's row: 32 bf16
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const uint4 v4 = ld_shared_v4(stg + sidx(lane, c));
+          xr[4 * c] = v4.x;
+          xr[4 * c + 1] = v4.y;
+          xr[4 * c + 2] = v4.z;
+          xr[4 * c + 3] = v4.w;
+        }
         const float c2t = ms->c2[cb][t];
         const float et = ex2(c2t);
         const float ut = ms->steep[cb] ? 1.f : ex2(c2t - ms->c2ref[cb]);
         const float Dh = D[h];
-        const uint32_t acc = tmem + lane_off + TM_ACC + 128u * s;
-        const int rbase = t0 + 128 * ti + 32 * q;  // first (chunk-absolute) row of this warp
-        float *ybase = y + (((size_t)bi * d.L + rbase) * d.H + h) * TP;
-        const size_t yrow_stride = (size_t)d.H * TP;
+        tmem_ld_wait();
+        __syncwarp();
+        float *yw = y + (((size_t)bi * d.L + t0 + row0) * d.H + h) * TP + 32 * hf;
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          float vi[32], va[32];
-          tmem_ld32(acc + 32u * half, vi);
-          tmem_ld32(acc + 64u + 32u * half, va);
-          tmem_ld_wait();
+        for (int pass = 0; pass < 2; ++pass) {  // channels 16 pass .. 16 pass + 15 of the half
 #pragma unroll
-          for (int cc = 0; cc < 8; ++cc) {  // 8 chunks of 4 fp32 = the 32 channels of this half
-            const uint4 xw = xg[4 * half + cc / 2];
-            const uint32_t w0 = (cc & 1) ? xw.z : xw.x, w1 = (cc & 1) ? xw.w : xw.y;
-            const float xv[4] = {__uint_as_float(w0 << 16), __uint_as_float(w0 & 0xffff0000u),
-                                 __uint_as_float(w1 << 16), __uint_as_float(w1 & 0xffff0000u)};
+          for (int c = 0; c < 4; ++c) {
             float o[4];
 #pragma unroll
-            for (int m = 0; m < 4; ++m) o[m] = fmaf(et, vi[4 * cc + m], fmaf(ut, va[4 * cc + m], Dh * xv[m]));
-            st_shared_v4(stg + (uint32_t)lane * 128u + ((cc ^ (lane & 7)) << 4), __float_as_uint(o[0]),
-                         __float_as_uint(o[1]), __float_as_uint(o[2]), __float_as_uint(o[3]));
+            for (int m = 0; m < 4; ++m) {
+              const int e = 16 * pass + 4 * c + m;
+              const uint32_t wv = xr[e >> 1];
+              const float xv = __uint_as_float((e & 1) ? (wv & 0xffff0000u) : (wv << 16));
+              o[m] = fmaf(et, vi[e], fmaf(ut, va[e], Dh * xv));
+            }
+            st_shared_v4(stg + sidx(lane, c), __float_as_uint(o[0]), __float_as_uint(o[1]), __float_as_uint(o[2]),
+                         __float_as_uint(o[3]));
           }
           __syncwarp();
 #pragma unroll
-          for (int it = 0; it < 8; ++it) {  // rows 4*it .. 4*it+3 of the warp, 8 threads per row
-            const int rr = 4 * it + (lane >> 3), cc = lane & 7;
-            const uint4 v = ld_shared_v4(stg + (uint32_t)rr * 128u + ((cc ^ (rr & 7)) << 4));
-            if (128 * ti + 32 * q + rr < valid)
-              *reinterpret_cast<uint4 *>(ybase + (size_t)rr * yrow_stride + 32 * half + 4 * cc) = v;
+          for (int it = 0; it < 4; ++it) {
+            const int rr = 8 * it + (lane >> 2), c = lane & 3;
+            const uint4 v4 = ld_shared_v4(stg + sidx(rr, c));
+            if (rr < nrows) *reinterpret_cast<uint4 *>(yw + (size_t)rr * rstride + 16 * pass + 4 * c) = v4;
           }
           __syncwarp();
         }
       }
       tc_fence_before();
-      named_barrier(2, 128);
+      named_barrier(2, 256);
       if (tid == 0 && ok) {
         mbar_arrive(&ms->acc_free[s]);
         mbar_arrive(&ms->cum_free[cb]);
