@@ -213,29 +213,47 @@ def prefill_work(w, Q=None):
 
 
 def kernel_work(name, w, Q):
-    """(bound, algorithmic amount per launch, unit) of one prefill kernel."""
+    """(bound, algorithmic amount per launch, unit, flops per launch) of one prefill kernel.
+
+    Bytes are what the kernel must move given the pipeline's intermediates: the chunk
+    states S (fp32, written by chunk_state, read by state passing) and the state entering
+    each chunk (bf16, written by state passing, read by chunk_scan)."""
     b, L, H, P, N, G = w.batch, w.seqlen, w.nheads, w.headdim, w.dstate, w.ngroups
     tok, nc = b * L, -(-w.seqlen // Q)
     el = 2 if w.dtype == "bf16" else 4
+    x_b, bc_b, dt_b = tok * H * P * el, tok * G * N * el, tok * H * 4
+    states = b * nc * H * P * N
+    flops_state = tok * H * 2 * N * P
+    flops_scan = tok * H * (2 * Q * P + 2 * N * P) + tok * G * 2 * Q * N
     if name.startswith("dA_cumsum"):
-        return "hbm", tok * H * 4 + b * H * nc * Q * 4, "bytes"
+        return "hbm", dt_b + b * H * nc * Q * 4, "bytes", 0
+    if name == "state_passing":
+        return "hbm", 2 * states * 4 + b * H * P * N * 4, "bytes", 0
     if name.startswith("state_passing"):
-        return "hbm", 2 * b * nc * H * P * N * 4 + b * H * P * N * 4, "bytes"
+        return "hbm", states * 4 + states * 2 + b * H * P * N * 4 + b * H * nc * 4, "bytes", 0
+    if name == "chunk_state_tc":
+        return "hbm", x_b + bc_b + dt_b + states * 4 + b * H * nc * 4, "bytes", flops_state
+    if name == "chunk_scan_tc":
+        return "hbm", x_b + 2 * bc_b + dt_b + states * 2 + tok * H * P * 4, "bytes", flops_scan
     if name.startswith("chunk_state"):
-        return "flops", tok * H * 2 * N * P, "flops"
+        return "flops", flops_state, "flops", flops_state
     if name.startswith("chunk_scan"):
-        return "flops", tok * H * (2 * Q * P + 2 * N * P) + tok * G * 2 * Q * N, "flops"
-    return "hbm", 0, "bytes"
+        return "flops", flops_scan, "flops", flops_scan
+    return "hbm", 0, "bytes", 0
 
 
 def roofline_entry(name, w, Q, avg_ms, peaks, traffic):
-    kind, amount, _ = kernel_work(name, w, Q)
+    kind, amount, _, flops = kernel_work(name, w, Q)
     secs = avg_ms / 1e3
     if kind == "hbm":
         achieved = amount / secs / 1e9
-        return {"kernel": name, "bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": achieved / peaks["hbm_gbs"], "traffic": traffic,
-                "peak_source": f"{peaks['source']} hbm_gbs"}
+        e = {"kernel": name, "bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+             "frac": achieved / peaks["hbm_gbs"], "traffic": traffic, "algorithmic_bytes": amount,
+             "peak_source": f"{peaks['source']} hbm_gbs"}
+        if flops:
+            e["tensor_tflops"] = flops / secs / 1e12
+            e["tensor_frac"] = flops / secs / 1e12 / peaks["bf16_tflops"]
+        return e
     achieved = amount / secs / 1e12
     if name.endswith("_simt"):  # fp32 FMA on CUDA cores
         return {"kernel": name, "bound": "alu", "achieved": achieved, "peak": FP32_SIMT_PEAK_TFLOPS,
@@ -352,7 +370,6 @@ def prefill_leg(args, dev, rank, world, peaks, sampler):
     avg = {n: statistics.mean(kern_ms[i]) for i, n in enumerate(names)}
     tot = sum(avg.values())
     dom = max(avg, key=avg.get)
-    kernel_srcs = {n: ["selective_state_space_10_b200/csrc/prefill_simt.cu"] for n in names}
     res = {
         "value": value, "ms_per_step": ms_per_step, "tokens_per_step_per_gpu": tokens,
         "tflops": {"dense_tile": fl_dense / secs / 1e12, "causal_only": fl_causal / secs / 1e12,
@@ -360,7 +377,9 @@ def prefill_leg(args, dev, rank, world, peaks, sampler):
                    "peak": peaks["bf16_tflops"], "peak_source": f"{peaks['source']} bf16_tflops (burst)"},
         "hbm": {"min_bytes": min_bytes, "GB/s": min_bytes / secs / 1e9,
                 "frac": min_bytes / secs / 1e9 / peaks["hbm_gbs"], "peak": peaks["hbm_gbs"]},
-        "kernels": {n: {"avg_ms": avg[n], "share": avg[n] / tot} for n in names},
+        "kernels": {n: {"avg_ms": avg[n], "share": avg[n] / tot,
+                        "roofline": roofline_entry(n, w, w.chunk, avg[n], peaks, profile_traffic(n, w.name))}
+                    for n in names},
         "roofline": roofline_entry(dom, w, w.chunk, avg[dom], peaks, profile_traffic(dom, w.name)),
         "gpu_launches": K * nk,
         "config": {"workload": w.name, "batch": w.batch, "seqlen": w.seqlen, "nheads": w.nheads,
@@ -369,7 +388,6 @@ def prefill_leg(args, dev, rank, world, peaks, sampler):
                    "l2": "256 MiB buffer written before every timed step (not timed): inputs fit in L2",
                    "parallelism": f"{world} GPU(s), one independent sequence per GPU, no collective"},
     }
-    _ = kernel_srcs
     # End to end: pinned host inputs -> device, prefill, y and final state -> pinned host.
     host = {k: v.cpu().pin_memory() for k, v in t.items()}
     y_h = torch.empty(y.shape, dtype=y.dtype, pin_memory=True)
