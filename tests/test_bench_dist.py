@@ -1,0 +1,79 @@
+"""bench.py's multi-process plumbing on CPU (gloo, world size 2) and its work model.
+
+The timed GPU legs need a B200; what runs per rank around them -- process-group set-up,
+barriers, the max-over-ranks reduction of the timed region, per-rank seeds (every rank
+runs its own independent sequence: weak scaling, no collective on the data path) and the
+reference arm's rank-0-only rule -- is exercised here with real processes."""
+import os
+import socket
+
+import pytest
+import torch.multiprocessing as mp
+
+import bench
+from selective_state_space_10_b200 import inputs
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world),
+                      LOCAL_RANK=str(rank))
+    import torch
+    assert bench.dist_env() == (rank, world, rank)
+    dist = bench.init_dist(world, "gloo")
+    bench.barrier(world)
+    t_max = bench.max_over_ranks(10.0 + rank, world, torch.device("cpu"))
+    seed = bench.rank_seed(inputs.BY_NAME["mamba2_2.7b_prefill"].seed, rank)
+    seeds = [None] * world
+    dist.all_gather_object(seeds, seed)
+    # the reference arm: ranks other than 0 leave at once, without work
+    rc = bench.run_reference(type("A", (), {"workload": "mamba2_2.7b_prefill", "steps": 1, "warmup": 3})()) \
+        if rank != 0 else 0
+    bench.barrier(world)
+    dist.destroy_process_group()
+    out.put((rank, t_max, seeds, rc))
+
+
+def test_two_ranks_gloo():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = [q.get(timeout=120) for _ in procs]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    res.sort()
+    for rank, t_max, seeds, rc in res:
+        assert t_max == 11.0            # the slowest rank's time is the job's time
+        assert len(set(seeds)) == 2     # independent sequences per rank
+        assert rc == 0
+    assert res[0][2] == res[1][2]
+
+
+def test_work_model_matches_the_hand_computed_budgets():
+    """Dense-tile FLOPs and minimum bytes of the 2.7B- and 130M-shaped prefills."""
+    w2 = inputs.BY_NAME["mamba2_2.7b_prefill"]
+    dense, causal, min_bytes = bench.prefill_work(w2)
+    assert dense == pytest.approx(21.74e9, rel=2e-3)
+    assert causal == pytest.approx(16.26e9, rel=2e-3)
+    # x, B, C bf16 + dt + A, D in; y fp32 + final state out
+    assert min_bytes == 4096 * 80 * 64 * 2 + 2 * 4096 * 128 * 2 + 4096 * 80 * 4 + 2 * 80 * 4 \
+        + 4096 * 80 * 64 * 4 + 80 * 64 * 128 * 4
+    w1 = inputs.BY_NAME["mamba2_130m_prefill"]
+    assert bench.prefill_work(w1)[0] == pytest.approx(6.71e9, rel=3e-3)
+
+
+def test_kernel_work_is_below_the_ridge_for_the_tensor_core_kernels():
+    w = inputs.BY_NAME["mamba2_2.7b_prefill"]
+    for name in ("chunk_state_tc", "chunk_scan_tc"):
+        kind, nbytes, _, flops = bench.kernel_work(name, w, w.chunk)
+        assert kind == "hbm" and nbytes > 0
+        assert flops / nbytes < 1657.6e12 / 6539.2e9  # arithmetic intensity below the ridge
