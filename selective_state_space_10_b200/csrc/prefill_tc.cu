@@ -40,6 +40,15 @@
 #include <cuda_bf16.h>
 #include <stddef.h>
 
+#include <algorithm>
+#include <cmath>
+#include <functional>
+#include <map>
+#include <mutex>
+#include <queue>
+#include <tuple>
+#include <vector>
+
 #include "common.cuh"
 #include "kernels.h"
 #include "sm100.cuh"
@@ -382,22 +391,24 @@ k_chunk_scan_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                 const __grid_constant__ CUtensorMap tm_B, const __grid_constant__ CUtensorMap tm_h,
                 const __nv_bfloat16 *__restrict__ x, const float *__restrict__ dt, const float *__restrict__ A,
                 const float *__restrict__ D, float *__restrict__ y, int *err,
-                Dims d, int Q, int nc, int kb, int nhb) {
+                Dims d, int Q, int nc, int kb0, int nhb0, int kb1, int nhb1) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   K3Misc *ms = reinterpret_cast<K3Misc *>(base + K3Smem::misc);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int ntt = Q / 128;
 
+  // work item: (bi, c, g, j); j < nhb1 are the second row tile's head blocks (the heavier
+  // CTAs, scheduled first), the rest the first tile's
   int item = blockIdx.x;
-  const int hb = item % nhb;
-  item /= nhb;
+  const int j = item % (nhb0 + nhb1);
+  item /= nhb0 + nhb1;
   const int g = item % d.G;
   item /= d.G;
-  const int ti = item % ntt;  // 128-row token tile inside the chunk
-  item /= ntt;
   const int c = item % nc;
   const int bi = item / nc;
+  const int ti = (j < nhb1) ? 1 : 0;  // 128-row token tile inside the chunk
+  const int hb = (j < nhb1) ? j : j - nhb1;
+  const int kb = ti ? kb1 : kb0;
   const int h0 = g * d.hpg + hb * kb;
   const int nh = min(kb, d.hpg - hb * kb);
   const int t0 = c * Q;
@@ -808,6 +819,55 @@ int pick_heads_per_cta(int base_items, int hpg, int sms, double overhead) {
   return best_kb;
 }
 
+// Head split of the chunk-scan kernel.  A CTA of the second row tile costs about 1.5x a
+// first-tile CTA per head (twice the x tile and the in-chunk product); each also pays a
+// fixed set-up (about 1.8 heads).  Candidate splits are scored by simulating the
+// hardware's greedy, in-order placement of CTAs onto SMs (one CTA per SM at a time).
+struct ScanSplit {
+  int kb0, nhb0, kb1, nhb1;
+};
+
+double simulate_makespan(int groups, int hpg, int kb0, int kb1, int ntt, int sms) {
+  constexpr double kSetup = 1.8, kTile1 = 1.5;
+  std::vector<double> free_at(sms, 0.0);
+  std::priority_queue<double, std::vector<double>, std::greater<double>> q(free_at.begin(), free_at.end());
+  const int nhb0 = (hpg + kb0 - 1) / kb0, nhb1 = ntt > 1 ? (hpg + kb1 - 1) / kb1 : 0;
+  double end = 0.0;
+  for (int gi = 0; gi < groups; ++gi)
+    for (int jj = 0; jj < nhb0 + nhb1; ++jj) {
+      const bool t1 = jj < nhb1;
+      const int kb = t1 ? kb1 : kb0, hb = t1 ? jj : jj - nhb1;
+      const int nh = std::min(kb, hpg - hb * kb);
+      const double cost = kSetup + nh * (t1 ? kTile1 : 1.0);
+      const double start = q.top();
+      q.pop();
+      q.push(start + cost);
+      end = std::max(end, start + cost);
+    }
+  return end;
+}
+
+ScanSplit pick_scan_split(int groups, int hpg, int ntt, int sms) {
+  static std::mutex mu;
+  static std::map<std::tuple<int, int, int, int>, ScanSplit> cache;
+  const auto key = std::make_tuple(groups, hpg, ntt, sms);
+  std::lock_guard<std::mutex> lock(mu);
+  auto it = cache.find(key);
+  if (it != cache.end()) return it->second;
+  ScanSplit best{hpg, 1, hpg, ntt > 1 ? 1 : 0};
+  double best_t = 1e300;
+  for (int kb1 = 1; kb1 <= hpg; ++kb1) {
+    const int kb0 = ntt > 1 ? std::min(hpg, std::max(1, (int)std::lround(kb1 * 1.5))) : kb1;
+    const double t = simulate_makespan(groups, hpg, kb0, kb1, ntt, sms);
+    if (t < best_t - 1e-9) {
+      best_t = t;
+      best = {kb0, (hpg + kb0 - 1) / kb0, kb1, ntt > 1 ? (hpg + kb1 - 1) / kb1 : 0};
+    }
+  }
+  cache[key] = best;
+  return best;
+}
+
 }  // namespace
 
 bool tc_prefill_supported(const Dims &d, int Q) { return d.P == TP && d.N == TN && (Q == 128 || Q == 256); }
@@ -854,13 +914,12 @@ cudaError_t launch_tc_prefill(const __nv_bfloat16 *x, const float *dt, const flo
   // K3
   {
     const int ntt = Q / 128;
-    const int base_items = d.b * nc * ntt * d.G;
-    const int kb = pick_heads_per_cta(base_items, d.hpg, sms, 2.0);
-    const int nhb = (d.hpg + kb - 1) / kb;
+    const int groups = d.b * nc * d.G;
+    const ScanSplit sp = pick_scan_split(groups, d.hpg, ntt, sms);
     e = cudaFuncSetAttribute(k_chunk_scan_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kK3SmemBytes);
     if (e != cudaSuccess) return e;
-    k_chunk_scan_tc<<<(unsigned)(base_items * nhb), K3_THREADS, kK3SmemBytes, st>>>(
-        tm_x3, tm_C3, tm_B3, tm_h3, x, dt, A, D, y, err, d, Q, nc, kb, nhb);
+    k_chunk_scan_tc<<<(unsigned)(groups * (sp.nhb0 + sp.nhb1)), K3_THREADS, kK3SmemBytes, st>>>(
+        tm_x3, tm_C3, tm_B3, tm_h3, x, dt, A, D, y, err, d, Q, nc, sp.kb0, sp.nhb0, sp.kb1, sp.nhb1);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   return mark(3);
