@@ -47,6 +47,7 @@
 #include <mutex>
 #include <queue>
 #include <tuple>
+#include <utility>
 #include <vector>
 
 #include "common.cuh"
@@ -107,6 +108,7 @@ k_chunk_state_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
   const int nh = min(kb, d.hpg - hb * kb);
   const int t0 = c * Q;
   const int valid = min(Q, d.L - t0);
+  grid_dep_launch();  // state passing may be scheduled now; it waits for this grid's results
 
   if (threadIdx.x == 0) {
     mbar_init(&ms->b_full, 1);
@@ -299,6 +301,8 @@ k_state_passing_bf16(const float *__restrict__ states, const float *__restrict__
                      __nv_bfloat16 *__restrict__ hprev, float *__restrict__ final_state, Dims d, int nc) {
   const int PN4 = d.P * d.N / 4;
   const int e4 = blockIdx.y * blockDim.x + threadIdx.x;
+  sm100::grid_dep_launch();  // the chunk scan may start its own set-up meanwhile
+  sm100::grid_dep_wait();    // chunk states and decays of the chunk-state kernel
   if (e4 >= PN4) return;
   const int h = blockIdx.x % d.H, bi = blockIdx.x / d.H;
   const size_t cstride = (size_t)d.H * PN4;  // float4s between consecutive chunks
@@ -458,13 +462,24 @@ k_chunk_scan_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
         for (int kn = 0; kn < 2; ++kn)
           tma_load_3d(base + K3Smem::bw + (uint32_t)kn * nblk * 16384u + j * 16384u, &tm_B, &ms->cb_full,
                       g * TN + 64 * kn, t0 + 128 * j, bi);
+      // x of the first two heads is an input: fetch it before waiting for the state-passing
+      // kernel, whose chunk-start states (h) are the only thing read from it
+      const int pre = min(nh, 2);
+      for (int k = 0; k < pre; ++k) {
+        mbar_arrive_expect_tx(&ms->x_full[k], (uint32_t)nblk * 16384u + 16384u);
+        for (int j = 0; j < nblk; ++j)
+          tma_load_3d(base + K3Smem::x(k) + j * 16384u, &tm_x, &ms->x_full[k], (h0 + k) * TP, t0 + 128 * j, bi);
+      }
+      grid_dep_wait();
       int issued = 0;
       for (int k = 0; k < nh; ++k) {
         const int s = k & 1, u = k >> 1, h = h0 + k;
-        if (k >= 2 && !mbar_wait(&ms->x_free[s], (u - 1) & 1, abort_flag, err)) break;
-        mbar_arrive_expect_tx(&ms->x_full[s], (uint32_t)nblk * 16384u + 16384u);
-        for (int j = 0; j < nblk; ++j)
-          tma_load_3d(base + K3Smem::x(s) + j * 16384u, &tm_x, &ms->x_full[s], h * TP, t0 + 128 * j, bi);
+        if (k >= pre) {
+          if (!mbar_wait(&ms->x_free[s], (u - 1) & 1, abort_flag, err)) break;
+          mbar_arrive_expect_tx(&ms->x_full[s], (uint32_t)nblk * 16384u + 16384u);
+          for (int j = 0; j < nblk; ++j)
+            tma_load_3d(base + K3Smem::x(s) + j * 16384u, &tm_x, &ms->x_full[s], h * TP, t0 + 128 * j, bi);
+        }
         for (int kn = 0; kn < 2; ++kn)
           tma_load_3d(base + K3Smem::hs(s) + kn * 8192u, &tm_h, &ms->x_full[s], 64 * kn, 0, (bi * nc + c) * d.H + h);
         issued = k + 1;
@@ -868,6 +883,24 @@ ScanSplit pick_scan_split(int groups, int hpg, int ntt, int sms) {
   return best;
 }
 
+// Launch `kern` on `st`; with `pdl` it may begin while the previous kernel in the stream is
+// still running, and must call grid_dep_wait() before it reads that kernel's results.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_after(dim3 grid, unsigned threads, size_t smem, cudaStream_t st, bool pdl,
+                         void (*kern)(KArgs...), Args &&...args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(threads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
 }  // namespace
 
 bool tc_prefill_supported(const Dims &d, int Q) { return d.P == TP && d.N == TN && (Q == 128 || Q == 256); }
@@ -888,6 +921,9 @@ cudaError_t launch_tc_prefill(const __nv_bfloat16 *x, const float *dt, const flo
     return cudaErrorInvalidValue;
   const int sms = num_sms();
   auto mark = [&](int i) { return ev ? cudaEventRecord(ev[i], st) : cudaSuccess; };
+  // Without per-kernel events the three kernels overlap their set-up with the tail of the
+  // one before (programmatic dependent launch); with events between them they run serially.
+  const bool pdl = ev == nullptr;
   cudaError_t e = mark(0);
   if (e != cudaSuccess) return e;
   // K1
@@ -906,9 +942,9 @@ cudaError_t launch_tc_prefill(const __nv_bfloat16 *x, const float *dt, const flo
   // K2
   {
     const int per_head = d.P * d.N / 4;
-    k_state_passing_bf16<<<dim3(d.b * d.H, (per_head + 255) / 256), 256, 0, st>>>(states, cdecay, hprev, final_state,
-                                                                                 d, nc);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    e = launch_after(dim3(d.b * d.H, (per_head + 255) / 256), 256, 0, st, pdl, k_state_passing_bf16, states, cdecay,
+                     hprev, final_state, d, nc);
+    if (e != cudaSuccess) return e;
   }
   if ((e = mark(2)) != cudaSuccess) return e;
   // K3
@@ -918,9 +954,10 @@ cudaError_t launch_tc_prefill(const __nv_bfloat16 *x, const float *dt, const flo
     const ScanSplit sp = pick_scan_split(groups, d.hpg, ntt, sms);
     e = cudaFuncSetAttribute(k_chunk_scan_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kK3SmemBytes);
     if (e != cudaSuccess) return e;
-    k_chunk_scan_tc<<<(unsigned)(groups * (sp.nhb0 + sp.nhb1)), K3_THREADS, kK3SmemBytes, st>>>(
-        tm_x3, tm_C3, tm_B3, tm_h3, x, dt, A, D, y, err, d, Q, nc, sp.kb0, sp.nhb0, sp.kb1, sp.nhb1);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    e = launch_after(dim3((unsigned)(groups * (sp.nhb0 + sp.nhb1))), K3_THREADS, kK3SmemBytes, st, pdl,
+                     k_chunk_scan_tc, tm_x3, tm_C3, tm_B3, tm_h3, x, dt, A, D, y, err, d, Q, nc, sp.kb0, sp.nhb0,
+                     sp.kb1, sp.nhb1);
+    if (e != cudaSuccess) return e;
   }
   return mark(3);
 }
