@@ -343,29 +343,46 @@ k_state_passing_bf16(const float *__restrict__ states, const float *__restrict__
 // row factor u_t = 2^(c2_t - c2_r) and a column factor v_s = 2^(c2_r - c2_s) dt_s.  Hence
 //     sum_s W_ts x_s = u_t * sum_s (G o mask)_ts (v_s x_s),
 // where G o mask (causal) does not depend on the head: it is converted to bf16 once per
-// CTA (W_base), and each head only scales the rows of its x tile by v_s.  This is exact
-// algebra; it is used when the tile's decay range |c2_r - c2_last| is below 100 (then
-// every factor lies in [2^-100, 2^100] and all intermediates stay normal fp32).  Heads
-// with a steeper tile ("steep" heads) build their own W with per-32-token references
+// CTA (W_base, kept in TMEM as the A operand of the intra-chunk MMA), and each head only
+// scales the rows of its x tile by v_s.  This is exact algebra; it is used when the
+// tile's decay range |c2_r - c2_last| is below 100 (then every factor lies in
+// [2^-100, 2^100] and all intermediates stay normal fp32).  Heads with a steeper tile
+// ("steep" heads) get their own W (W_base times the full decay, in a second TMEM region)
 // instead, as a slower exact fallback.
+//
+// With W in TMEM, shared memory holds only the C tile, the output staging and a ring of
+// per-head slots (x tile + h_prev^T): 5 slots for the first row tile, 3 for the second,
+// so that several heads' loads are in flight while earlier heads are scaled and stored.
 constexpr int K3_THREADS = 480;  // warp 0 TMA, 1 MMA, 2-5 W/x scaling, 6-13 output, 14 decay tables
 constexpr int K3_CUMBUF = 3;
+constexpr int K3_MAXSLOTS = 5;
 constexpr float kSteepLog2 = 100.f;
 
 struct K3Smem {
-  static constexpr uint32_t cm = 0;      // C tile: 2 K-atoms x [128][128 B]                          32 KB
-  static constexpr uint32_t bw = 32768;  // B rows (for G), then W (W_base or a steep head's W)       64 KB
-  // x tiles: nblk blocks of [128 rows][128 B]; after the head's MMAs, y staging (2 x [128][128 B])
-  __host__ __device__ static constexpr uint32_t x(int s) { return 98304u + (uint32_t)s * 32768u; }  // 2 x 32 KB
-  __host__ __device__ static constexpr uint32_t hs(int s) { return 163840u + (uint32_t)s * 16384u; } // 2 x 16 KB
+  static constexpr uint32_t cm = 0;  // C tile: 2 K-atoms x [128][128 B]                                32 KB
   // x/y staging: one [32 rows][64 B] buffer per output warp (8 x 2 KB)
-  __host__ __device__ static constexpr uint32_t ystage(int w) { return 196608u + (uint32_t)w * 2048u; }
-  static constexpr uint32_t misc = 212992u;
+  __host__ __device__ static constexpr uint32_t ystage(int w) { return 32768u + (uint32_t)w * 2048u; }
+  static constexpr uint32_t misc = 49152u;  // K3Misc, at most 10 KB
+  static constexpr uint32_t ring = 59392u;  // slot ring; the B rows for G sit at its end until G is formed
+  static constexpr uint32_t end = 231424u;  // 227 KB of dynamic shared memory less the alignment slack
+  // slot: nblk x blocks of [128 rows][128 B], then h_prev^T as 2 K-halves of [64][128 B]
+  __host__ __device__ static constexpr uint32_t slot_bytes(int nblk) { return (uint32_t)nblk * 16384u + 16384u; }
+  __host__ __device__ static constexpr int slots(int nblk) {
+    return (end - ring) / slot_bytes(nblk) < (uint32_t)K3_MAXSLOTS ? (int)((end - ring) / slot_bytes(nblk))
+                                                                    : K3_MAXSLOTS;
+  }
+  __host__ __device__ static constexpr uint32_t slot(int nblk, int s) { return ring + (uint32_t)s * slot_bytes(nblk); }
+  // B rows for G: 2 K-atoms, each [128 * nblk rows][128 B]
+  __host__ __device__ static constexpr uint32_t bm(int nblk) { return end - (uint32_t)nblk * 32768u; }
 };
+static_assert(K3Smem::slots(1) == 5 && K3Smem::slots(2) == 3, "slot ring depth");
+static_assert(K3Smem::ring % 1024 == 0 && K3Smem::bm(1) % 1024 == 0 && K3Smem::bm(2) % 1024 == 0,
+              "TMA destinations with 128-byte swizzle must be 1024-byte aligned");
 
 struct K3Misc {
-  uint64_t cb_full, g_full;
-  uint64_t x_full[2], ops_ready[2], x_free[2], acc_full[2], acc_free[2];
+  uint64_t cb_full, g_full, w_ready;
+  uint64_t x_full[K3_MAXSLOTS], ops_ready[K3_MAXSLOTS], x_free[K3_MAXSLOTS];
+  uint64_t acc_full[2], acc_free[2];
   uint64_t cum_full[K3_CUMBUF], cum_free[K3_CUMBUF];
   uint32_t tmem;
   int abort_flag;
@@ -378,17 +395,14 @@ struct K3Misc {
 };
 static_assert(offsetof(K3Misc, c2) % 16 == 0 && offsetof(K3Misc, v) % 16 == 0, "decay tables must be 16-byte aligned");
 static_assert(K3Smem::misc % 16 == 0, "K3Misc must start 16-byte aligned");
+static_assert(K3Smem::misc + sizeof(K3Misc) <= K3Smem::ring, "K3Misc overlaps the slot ring");
 
-constexpr size_t kK3SmemBytes = 1024 + K3Smem::misc + sizeof(K3Misc);
+constexpr size_t kK3SmemBytes = 1024 + K3Smem::end;
 
-// Writes 32 bf16 (packed pairs) into a K-major 128B-swizzled row: chunks cc0..cc0+3.
-__device__ __forceinline__ void st_row_bf16(uint32_t row_addr, int row, int cc0, const float *g) {
-#pragma unroll
-  for (int cc = 0; cc < 4; ++cc)
-    st_shared_v4(row_addr + (((cc0 + cc) ^ (row & 7)) << 4), pack_bf16x2(g[8 * cc + 0], g[8 * cc + 1]),
-                 pack_bf16x2(g[8 * cc + 2], g[8 * cc + 3]), pack_bf16x2(g[8 * cc + 4], g[8 * cc + 5]),
-                 pack_bf16x2(g[8 * cc + 6], g[8 * cc + 7]));
-}
+// TMEM columns: W_base and a steep head's W (bf16 pairs, 64 columns per 128-token block),
+// then two accumulator slots of [inter 64 | intra 64] columns.  G (fp32, 128 * nblk
+// columns) occupies the accumulator slots until W_base has been built from it.
+constexpr uint32_t K3_TM_WB = 0, K3_TM_WS = 128, K3_TM_ACC = 256;
 
 __global__ void __launch_bounds__(K3_THREADS, 1)
 k_chunk_scan_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_C,
@@ -401,17 +415,17 @@ k_chunk_scan_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
   K3Misc *ms = reinterpret_cast<K3Misc *>(base + K3Smem::misc);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  // work item: (bi, c, g, j); j < nhb1 are the second row tile's head blocks (the heavier
+  // work item: (bi, c, g, jb); jb < nhb1 are the second row tile's head blocks (the heavier
   // CTAs, scheduled first), the rest the first tile's
   int item = blockIdx.x;
-  const int j = item % (nhb0 + nhb1);
+  const int jb = item % (nhb0 + nhb1);
   item /= nhb0 + nhb1;
   const int g = item % d.G;
   item /= d.G;
   const int c = item % nc;
   const int bi = item / nc;
-  const int ti = (j < nhb1) ? 1 : 0;  // 128-row token tile inside the chunk
-  const int hb = (j < nhb1) ? j : j - nhb1;
+  const int ti = (jb < nhb1) ? 1 : 0;  // 128-row token tile inside the chunk
+  const int hb = (jb < nhb1) ? jb : jb - nhb1;
   const int kb = ti ? kb1 : kb0;
   const int h0 = g * d.hpg + hb * kb;
   const int nh = min(kb, d.hpg - hb * kb);
@@ -419,16 +433,21 @@ k_chunk_scan_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
   const int valid = min(Q, d.L - t0);
   if (ti * 128 >= valid) return;  // no rows of this tile exist (whole CTA, before any setup)
   const int nblk = ti + 1;        // source blocks j = 0..ti
+  const int NS = K3Smem::slots(nblk);
+  const uint32_t SB = K3Smem::slot_bytes(nblk);
 
   if (threadIdx.x == 0) {
     mbar_init(&ms->cb_full, 1);
     mbar_init(&ms->g_full, 1);
-    for (int s = 0; s < 2; ++s) {
+    mbar_init(&ms->w_ready, 1);
+    for (int s = 0; s < K3_MAXSLOTS; ++s) {
       mbar_init(&ms->x_full[s], 1);
       mbar_init(&ms->ops_ready[s], 1);
       mbar_init(&ms->x_free[s], 1);  // MMA commit
-      mbar_init(&ms->acc_full[s], 1);
-      mbar_init(&ms->acc_free[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&ms->acc_full[a], 1);
+      mbar_init(&ms->acc_free[a], 1);
     }
     for (int s = 0; s < K3_CUMBUF; ++s) {
       mbar_init(&ms->cum_full[s], 1);
@@ -446,7 +465,6 @@ k_chunk_scan_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
   tc_fence_after();
   const uint32_t tmem = ms->tmem;
   volatile int *abort_flag = &ms->abort_flag;
-  const uint32_t TM_G = 0, TM_ACC = 256;  // G: cols [0, 256); acc slot a: inter +128a, intra +128a+64
 
   if (warp == 0) {
     // ------------------------------------------------------------- TMA producer
@@ -455,65 +473,81 @@ k_chunk_scan_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
       tma_prefetch_desc(&tm_C);
       tma_prefetch_desc(&tm_B);
       tma_prefetch_desc(&tm_h);
+      const uint32_t bmo = K3Smem::bm(nblk);
       mbar_arrive_expect_tx(&ms->cb_full, 32768u + (uint32_t)nblk * 32768u);
       for (int kn = 0; kn < 2; ++kn)
         tma_load_3d(base + K3Smem::cm + kn * 16384u, &tm_C, &ms->cb_full, g * TN + 64 * kn, t0 + 128 * ti, bi);
-      for (int j = 0; j < nblk; ++j)
+      for (int jj = 0; jj < nblk; ++jj)
         for (int kn = 0; kn < 2; ++kn)
-          tma_load_3d(base + K3Smem::bw + (uint32_t)kn * nblk * 16384u + j * 16384u, &tm_B, &ms->cb_full,
-                      g * TN + 64 * kn, t0 + 128 * j, bi);
-      // x of the first two heads is an input: fetch it before waiting for the state-passing
-      // kernel, whose chunk-start states (h) are the only thing read from it
-      const int pre = min(nh, 2);
-      for (int k = 0; k < pre; ++k) {
-        mbar_arrive_expect_tx(&ms->x_full[k], (uint32_t)nblk * 16384u + 16384u);
-        for (int j = 0; j < nblk; ++j)
-          tma_load_3d(base + K3Smem::x(k) + j * 16384u, &tm_x, &ms->x_full[k], (h0 + k) * TP, t0 + 128 * j, bi);
+          tma_load_3d(base + bmo + (uint32_t)kn * nblk * 16384u + jj * 16384u, &tm_B, &ms->cb_full,
+                      g * TN + 64 * kn, t0 + 128 * jj, bi);
+      // x of the first heads is an input: fetch it before waiting for the state-passing
+      // kernel, whose chunk-start states (h) are the only thing read from it.  A slot that
+      // overlaps the B rows is filled only once G has been formed.
+      int pre = 0;
+      while (pre < min(nh, NS) && K3Smem::slot(nblk, pre) + SB <= bmo) {
+        mbar_arrive_expect_tx(&ms->x_full[pre], SB);
+        for (int jj = 0; jj < nblk; ++jj)
+          tma_load_3d(base + K3Smem::slot(nblk, pre) + jj * 16384u, &tm_x, &ms->x_full[pre], (h0 + pre) * TP,
+                      t0 + 128 * jj, bi);
+        ++pre;
       }
       grid_dep_wait();
+      bool g_seen = false;
       int issued = 0;
       for (int k = 0; k < nh; ++k) {
-        const int s = k & 1, u = k >> 1, h = h0 + k;
+        const int s = k % NS, u = k / NS, h = h0 + k;
+        const uint32_t so = K3Smem::slot(nblk, s);
         if (k >= pre) {
-          if (!mbar_wait(&ms->x_free[s], (u - 1) & 1, abort_flag, err)) break;
-          mbar_arrive_expect_tx(&ms->x_full[s], (uint32_t)nblk * 16384u + 16384u);
-          for (int j = 0; j < nblk; ++j)
-            tma_load_3d(base + K3Smem::x(s) + j * 16384u, &tm_x, &ms->x_full[s], h * TP, t0 + 128 * j, bi);
+          if (k >= NS) {
+            if (!mbar_wait(&ms->x_free[s], (u - 1) & 1, abort_flag, err)) break;
+          } else if (!g_seen) {
+            if (!(g_seen = mbar_wait(&ms->g_full, 0, abort_flag, err))) break;
+          }
+          mbar_arrive_expect_tx(&ms->x_full[s], SB);
+          for (int jj = 0; jj < nblk; ++jj)
+            tma_load_3d(base + so + jj * 16384u, &tm_x, &ms->x_full[s], h * TP, t0 + 128 * jj, bi);
         }
         for (int kn = 0; kn < 2; ++kn)
-          tma_load_3d(base + K3Smem::hs(s) + kn * 8192u, &tm_h, &ms->x_full[s], 64 * kn, 0, (bi * nc + c) * d.H + h);
+          tma_load_3d(base + so + (uint32_t)nblk * 16384u + kn * 8192u, &tm_h, &ms->x_full[s], 64 * kn, 0,
+                      (bi * nc + c) * d.H + h);
         issued = k + 1;
       }
       if (*abort_flag) {  // let this CTA's own loads land before it exits
         mbar_wait_drain(&ms->cb_full, 0);
-        for (int k = (issued > 2 ? issued - 2 : 0); k < issued; ++k) mbar_wait_drain(&ms->x_full[k & 1], (k >> 1) & 1);
+        for (int k = (issued > NS ? issued - NS : 0); k < issued; ++k) mbar_wait_drain(&ms->x_full[k % NS], (k / NS) & 1);
       }
     }
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      const uint32_t cm = smem_u32(base + K3Smem::cm), bw = smem_u32(base + K3Smem::bw);
+      const uint32_t cm = smem_u32(base + K3Smem::cm), bmm = smem_u32(base + K3Smem::bm(nblk));
       bool ok = mbar_wait(&ms->cb_full, 0, abort_flag, err);
       if (ok) {
         tc_fence_after();
+        // G = C_tile B^T: M = 128 rows, N = 128 * nblk source tokens, K = d_state
         const uint32_t idg = idesc_bf16_f32(128, 128 * nblk, false, false);
         for (int ks = 0; ks < 8; ++ks) {
           const uint64_t ad = smem_desc_sw128(cm + (ks >> 2) * 16384u + (ks & 3) * 32u, 16u, 1024u);
-          const uint64_t bd = smem_desc_sw128(bw + (ks >> 2) * (uint32_t)nblk * 16384u + (ks & 3) * 32u, 16u, 1024u);
-          mma_bf16(tmem + TM_G, ad, bd, idg, ks > 0 ? 1u : 0u);
+          const uint64_t bd = smem_desc_sw128(bmm + (ks >> 2) * (uint32_t)nblk * 16384u + (ks & 3) * 32u, 16u, 1024u);
+          mma_bf16(tmem + K3_TM_ACC, ad, bd, idg, ks > 0 ? 1u : 0u);
         }
         mma_commit(&ms->g_full);
       }
+      // G occupies the accumulator columns until W_base has been built from it
+      ok = ok && mbar_wait(&ms->w_ready, 0, abort_flag, err);
       const uint32_t id_inter = idesc_bf16_f32(128, TP, false, false);
       const uint32_t id_intra = idesc_bf16_f32(128, TP, false, true);
       for (int k = 0; ok && k < nh; ++k) {
-        const int s = k & 1, u = k >> 1;
+        const int s = k % NS, u = k / NS, a = k & 1, cb = k % K3_CUMBUF;
         if (!mbar_wait(&ms->x_full[s], u & 1, abort_flag, err)) break;
-        if (k >= 2 && !mbar_wait(&ms->acc_free[s], (u - 1) & 1, abort_flag, err)) break;
+        if (k >= 2 && !mbar_wait(&ms->acc_free[a], ((k >> 1) - 1) & 1, abort_flag, err)) break;
         tc_fence_after();
-        const uint32_t acc = tmem + TM_ACC + 128u * s;
-        const uint32_t hsa = smem_u32(base + K3Smem::hs(s));
+        const uint32_t acc = tmem + K3_TM_ACC + 128u * a;
+        const uint32_t so = smem_u32(base + K3Smem::slot(nblk, s));
+        const uint32_t hsa = so + (uint32_t)nblk * 16384u;
+        // ACC_inter = C_tile h_prev^T: K = d_state
         for (int ks = 0; ks < 8; ++ks) {
           const uint64_t ad = smem_desc_sw128(cm + (ks >> 2) * 16384u + (ks & 3) * 32u, 16u, 1024u);
           const uint64_t bd = smem_desc_sw128(hsa + (ks >> 2) * 8192u + (ks & 3) * 32u, 16u, 1024u);
@@ -521,86 +555,112 @@ k_chunk_scan_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
         }
         if (!mbar_wait(&ms->ops_ready[s], u & 1, abort_flag, err)) break;
         tc_fence_after();
-        const uint32_t xa = smem_u32(base + K3Smem::x(s));
-        for (int j = 0; j < nblk; ++j)
+        // ACC_intra = W X': A from TMEM (W_base, or the head's own W when steep), K = source tokens
+        const uint32_t wa = tmem + (ms->steep[cb] ? K3_TM_WS : K3_TM_WB);
+        for (int jj = 0; jj < nblk; ++jj)
           for (int ks = 0; ks < 8; ++ks) {
-            const uint64_t ad = smem_desc_sw128(bw + j * 32768u + (ks >> 2) * 16384u + (ks & 3) * 32u, 16u, 1024u);
-            const uint64_t bd = smem_desc_sw128(xa + j * 16384u + ks * 2048u, 16384u, 1024u);
-            mma_bf16(acc + 64, ad, bd, id_intra, (j > 0 || ks > 0) ? 1u : 0u);
+            const uint64_t bd = smem_desc_sw128(so + jj * 16384u + ks * 2048u, 16384u, 1024u);
+            mma_bf16_ts(acc + 64, wa + (uint32_t)(64 * jj + 8 * ks), bd, id_intra, (jj > 0 || ks > 0) ? 1u : 0u);
           }
-        mma_commit(&ms->acc_full[s]);
+        mma_commit(&ms->acc_full[a]);
         mma_commit(&ms->x_free[s]);
       }
     }
     __syncwarp();
   } else if (warp < 6) {
     // ------------------------------------------------------------- W build and x scaling (128 threads)
-    // W builds: thread (q, lane) owns row tl = 32q + lane of every source block, in four
-    // 32-column groups (the warp's rows are the 32-token group q of the tile).
+    // Thread (q, lane) owns row tl = 32q + lane of W (TMEM lane tl); the warp's rows are the
+    // 32-token group q of the tile.
     const int q = warp & 3;
     const int tl = q * 32 + lane;
     const int tid = threadIdx.x - 64;
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
     const int t = 128 * ti + tl;  // chunk-relative row
     const int r = 128 * ti - 1;   // reference token (tile start)
-    bool g_ready = false, w_is_base = false;
+    // W_base = G o causal mask in bf16, once
+    bool ok = mbar_wait(&ms->g_full, 0, abort_flag, err);
+    tc_fence_after();
+    if (ok) {
+      for (int jj = 0; jj < nblk; ++jj)
+        for (int grp = 0; grp < 4; ++grp) {
+          const int col0 = 128 * jj + 32 * grp;  // chunk-relative first source column
+          uint32_t pk[16];
+          if (jj == ti && grp > q) {  // strictly right of the diagonal
+#pragma unroll
+            for (int e = 0; e < 16; ++e) pk[e] = 0u;
+          } else {
+            float gg[32];
+            tmem_ld32(tmem + lane_off + K3_TM_ACC + (uint32_t)col0, gg);
+            tmem_ld_wait();
+            if (jj == ti && grp == q) {
+#pragma unroll
+              for (int e = 0; e < 32; ++e) gg[e] = (col0 + e <= t) ? gg[e] : 0.f;
+            }
+#pragma unroll
+            for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(gg[2 * e], gg[2 * e + 1]);
+          }
+          tmem_st16(tmem + lane_off + K3_TM_WB + (uint32_t)(64 * jj + 16 * grp), pk);
+        }
+      tmem_st_wait();
+    }
+    tc_fence_before();
+    named_barrier(1, 128);
+    if (tid == 0 && ok) mbar_arrive(&ms->w_ready);
     for (int k = 0; k < nh; ++k) {
-      const int cb = k % K3_CUMBUF, s = k & 1;
-      bool ok = mbar_wait(&ms->cum_full[cb], (k / K3_CUMBUF) & 1, abort_flag, err);
+      const int cb = k % K3_CUMBUF, s = k % NS;
+      ok = ok && mbar_wait(&ms->cum_full[cb], (k / K3_CUMBUF) & 1, abort_flag, err);
       const bool steep = ok && ms->steep[cb];
-      if (ok && (steep || !w_is_base)) {
-        // (re)build W: wait for every earlier MMA that reads the W region (the last is head k-1's)
-        if (k >= 1) ok = mbar_wait(&ms->x_free[(k - 1) & 1], ((k - 1) >> 1) & 1, abort_flag, err);
-        if (ok && !g_ready) ok = g_ready = mbar_wait(&ms->g_full, 0, abort_flag, err);
+      if (steep) {
+        // the head's own W, from W_base and the full decay; W_steep is free once the MMAs of
+        // head k-1 (the last that may have read it) are complete
+        if (k >= 1) ok = mbar_wait(&ms->x_free[(k - 1) % NS], ((k - 1) / NS) & 1, abort_flag, err);
         tc_fence_after();
         if (ok) {
           const float *c2 = ms->c2[cb];
+          const float *dts = ms->dts[cb];
           const float c2t = c2[t];
-          for (int j = 0; j < nblk; ++j) {
+          for (int jj = 0; jj < nblk; ++jj)
             for (int grp = 0; grp < 4; ++grp) {
-              // 32 columns = 64 bytes = chunks 4*(grp&1) .. +3 of K-atom grp>>1
-              const uint32_t wrow =
-                  smem_u32(base + K3Smem::bw) + j * 32768u + (uint32_t)(grp >> 1) * 16384u + (uint32_t)tl * 128u;
-              const int cc0 = 4 * (grp & 1);
-              float gg[32];
-              if (j == ti && grp > q) {  // strictly right of the diagonal
+              const int col0 = 128 * jj + 32 * grp;
+              uint32_t pk[16];
+              if (jj == ti && grp > q) {
 #pragma unroll
-                for (int e = 0; e < 32; ++e) gg[e] = 0.f;
+                for (int e = 0; e < 16; ++e) pk[e] = 0u;
               } else {
-                const int col0 = 128 * j + 32 * grp;  // chunk-relative first column
-                tmem_ld32(tmem + lane_off + TM_G + (uint32_t)col0, gg);
+                tmem_ld16u(tmem + lane_off + K3_TM_WB + (uint32_t)(64 * jj + 16 * grp), pk);
                 tmem_ld_wait();
-                if (!steep) {
-                  // W_base = G o causal mask
-                  if (j == ti && grp == q) {
+                float gg[32];
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) gg[e] = (col0 + e <= t) ? gg[e] : 0.f;
-                  }
-                } else if (j < ti) {
-                  const float u = ex2(c2t - c2[r]);
-                  const float *vf = ms->v[cb] + col0;  // reference r: the column factors of x scaling
+                for (int e = 0; e < 16; ++e) {
+                  gg[2 * e] = __uint_as_float(pk[e] << 16);
+                  gg[2 * e + 1] = __uint_as_float(pk[e] & 0xffff0000u);
+                }
+                if (jj < ti) {
+                  // an earlier block: the reference-token factors (both <= 1 for a decaying head)
+                  const float uf = ex2(c2t - c2[r]);
+                  const float *vf = ms->v[cb] + col0;
 #pragma unroll
-                  for (int e = 0; e < 32; ++e) gg[e] *= vf[e] * u;
+                  for (int e = 0; e < 32; ++e) gg[e] *= vf[e] * uf;
                 } else {
-                  // a steep head's own tile: one exp of a difference per element (never overflows)
-                  const float *dts = ms->dts[cb];
+                  // the tile's own block: one exp of a difference per element (never overflows)
 #pragma unroll
                   for (int e = 0; e < 32; ++e) {
-                    const int sidx = col0 + e;
-                    gg[e] = (sidx <= t) ? gg[e] * ex2(c2t - c2[sidx]) * dts[sidx] : 0.f;
+                    const int sx = col0 + e;
+                    gg[e] = (sx <= t) ? gg[e] * ex2(c2t - c2[sx]) * dts[sx] : 0.f;
                   }
                 }
+#pragma unroll
+                for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(gg[2 * e], gg[2 * e + 1]);
               }
-              st_row_bf16(wrow, tl, cc0, gg);
+              tmem_st16(tmem + lane_off + K3_TM_WS + (uint32_t)(64 * jj + 16 * grp), pk);
             }
-          }
-          w_is_base = !steep;
+          tmem_st_wait();
         }
       }
       // scale the rows of this head's x tile by v_s (not for steep heads: their W holds the decay)
-      ok = ok && mbar_wait(&ms->x_full[s], (k >> 1) & 1, abort_flag, err);
+      ok = ok && mbar_wait(&ms->x_full[s], (k / NS) & 1, abort_flag, err);
       if (ok && !steep) {
-        const uint32_t xs = smem_u32(base + K3Smem::x(s));
+        const uint32_t xs = smem_u32(base + K3Smem::slot(nblk, s));
         const float *vt = ms->v[cb];
         const int units = nblk * 128 * 8;  // 16-byte units: row = unit / 8 (rows of 128 B)
 #pragma unroll 4
@@ -641,7 +701,7 @@ k_chunk_scan_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
     // staging layout: 32 rows x 64 bytes, 16-byte chunk c of row r at (c ^ ((r >> 1) & 3))
     auto sidx = [](int rr, int c) -> uint32_t { return (uint32_t)rr * 64u + ((c ^ ((rr >> 1) & 3)) << 4); };
     for (int k = 0; k < nh; ++k) {
-      const int s = k & 1, cb = k % K3_CUMBUF, h = h0 + k;
+      const int a = k & 1, cb = k % K3_CUMBUF, h = h0 + k;
       // x rows of this warp (channels of its half), 4 threads per 64-byte row segment
       const size_t rstride = (size_t)d.H * TP;  // elements between consecutive tokens
       const __nv_bfloat16 *xw = x + (((size_t)bi * d.L + t0 + row0) * d.H + h) * TP + 32 * hf;
@@ -653,10 +713,10 @@ k_chunk_scan_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                               : make_uint4(0u, 0u, 0u, 0u);
       }
       bool ok = mbar_wait(&ms->cum_full[cb], (k / K3_CUMBUF) & 1, abort_flag, err);
-      ok = ok && mbar_wait(&ms->acc_full[s], (k >> 1) & 1, abort_flag, err);
+      ok = ok && mbar_wait(&ms->acc_full[a], (k >> 1) & 1, abort_flag, err);
       tc_fence_after();
       if (ok) {
-        const uint32_t acc = tmem + lane_off + TM_ACC + 128u * s + 32u * hf;
+        const uint32_t acc = tmem + lane_off + K3_TM_ACC + 128u * a + 32u * hf;
         float vi[32], va[32];
         tmem_ld32(acc, vi);
         tmem_ld32(acc + 64u, va);
@@ -710,7 +770,7 @@ k_chunk_scan_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
       tc_fence_before();
       named_barrier(2, 256);
       if (tid == 0 && ok) {
-        mbar_arrive(&ms->acc_free[s]);
+        mbar_arrive(&ms->acc_free[a]);
         mbar_arrive(&ms->cum_free[cb]);
       }
     }
