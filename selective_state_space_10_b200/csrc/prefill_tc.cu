@@ -251,17 +251,28 @@ k_chunk_state_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
     // ------------------------------------------------------------- decay-weight warp
     // w_t = exp(cum_end - cum_t) dt_t for each upcoming head (ring of K1_CUMBUF), and the
     // chunk's total decay exp(cum_end) for the state-passing kernel.
+    // dt and A of head k + 1 are loaded while head k's buffer is awaited and filled
     const int per = Q / 32;
-    for (int k = 0; k < nh; ++k) {
-      const int wb = k % K1_CUMBUF, h = h0 + k;
-      if (k >= K1_CUMBUF && !mbar_wait(&ms->w_free[wb], ((k / K1_CUMBUF) - 1) & 1, abort_flag, err)) break;
-      const float a2 = A[h] * kLog2e;
-      float c2[8], dtv[8];
-      float run = 0.f;
+    auto load_head = [&](int k, float (&v)[8], float &a) {
+      const int h = h0 + k;
+      a = A[h];
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
         const int t = lane * per + j;
-        dtv[j] = (j < per && t < valid) ? dt[((size_t)bi * d.L + t0 + t) * d.H + h] : 0.f;
+        v[j] = (j < per && t < valid) ? dt[((size_t)bi * d.L + t0 + t) * d.H + h] : 0.f;
+      }
+    };
+    float dtv[8], dtn[8], acur = 0.f, anxt = 0.f;
+    if (nh > 0) load_head(0, dtv, acur);
+    for (int k = 0; k < nh; ++k) {
+      const int wb = k % K1_CUMBUF, h = h0 + k;
+      if (k + 1 < nh) load_head(k + 1, dtn, anxt);
+      if (k >= K1_CUMBUF && !mbar_wait(&ms->w_free[wb], ((k / K1_CUMBUF) - 1) & 1, abort_flag, err)) break;
+      const float a2 = acur * kLog2e;
+      float c2[8];
+      float run = 0.f;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
         run += dtv[j] * a2;
         c2[j] = run;
       }
@@ -279,6 +290,9 @@ k_chunk_state_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
       if (lane == 0) cdecay[((size_t)bi * d.H + h) * nc + c] = ex2(cend);
       __syncwarp();
       if (lane == 0) mbar_arrive(&ms->w_full[wb]);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) dtv[j] = dtn[j];
+      acur = anxt;
     }
   }
 
@@ -776,17 +790,28 @@ k_chunk_scan_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
     }
   } else {
     // ------------------------------------------------------------- decay-table warp
+    // dt and A of head k + 1 are loaded while head k's buffer is awaited and filled
     const int per = Q / 32;
-    for (int k = 0; k < nh; ++k) {
-      const int cb = k % K3_CUMBUF, h = h0 + k;
-      if (k >= K3_CUMBUF && !mbar_wait(&ms->cum_free[cb], ((k / K3_CUMBUF) - 1) & 1, abort_flag, err)) break;
-      const float a2 = A[h] * kLog2e;
-      float c2v[8], dtv[8];
-      float run = 0.f;
+    auto load_head = [&](int k, float (&v)[8], float &a) {
+      const int h = h0 + k;
+      a = A[h];
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
         const int tt = lane * per + j;
-        dtv[j] = (j < per && tt < valid) ? dt[((size_t)bi * d.L + t0 + tt) * d.H + h] : 0.f;
+        v[j] = (j < per && tt < valid) ? dt[((size_t)bi * d.L + t0 + tt) * d.H + h] : 0.f;
+      }
+    };
+    float dtv[8], dtn[8], acur = 0.f, anxt = 0.f;
+    if (nh > 0) load_head(0, dtv, acur);
+    for (int k = 0; k < nh; ++k) {
+      const int cb = k % K3_CUMBUF;
+      if (k + 1 < nh) load_head(k + 1, dtn, anxt);
+      if (k >= K3_CUMBUF && !mbar_wait(&ms->cum_free[cb], ((k / K3_CUMBUF) - 1) & 1, abort_flag, err)) break;
+      const float a2 = acur * kLog2e;
+      float c2v[8];
+      float run = 0.f;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
         run += dtv[j] * a2;
         c2v[j] = run;
       }
@@ -818,6 +843,9 @@ k_chunk_scan_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&ms->cum_full[cb]);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) dtv[j] = dtn[j];
+      acur = anxt;
     }
   }
 
