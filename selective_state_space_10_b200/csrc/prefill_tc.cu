@@ -365,8 +365,12 @@ k_state_passing_bf16(const float *__restrict__ states, const float *__restrict__
 // instead, as a slower exact fallback.
 //
 // With W in TMEM, shared memory holds only the C tile, the output staging and a ring of
-// per-head slots (x tile + h_prev^T): 5 slots for the first row tile, 3 for the second,
+// per-head slots (x tile + h_prev^T): 4 slots for the first row tile, 3 for the second,
 // so that several heads' loads are in flight while earlier heads are scaled and stored.
+// The D x_t term enters through the accumulator: the scaling warps, which read every raw
+// x row anyway, store D x_t / u_t into the intra-chunk accumulator before the MMA adds
+// W X' onto it; the output warps then only combine the two accumulators and hand each
+// [32 rows][32 channels] tile of y to a TMA store.
 constexpr int K3_THREADS = 480;  // warp 0 TMA, 1 MMA, 2-5 W/x scaling, 6-13 output, 14 decay tables
 constexpr int K3_CUMBUF = 3;
 constexpr int K3_MAXSLOTS = 5;
@@ -374,10 +378,11 @@ constexpr float kSteepLog2 = 100.f;
 
 struct K3Smem {
   static constexpr uint32_t cm = 0;  // C tile: 2 K-atoms x [128][128 B]                                32 KB
-  // x/y staging: one [32 rows][64 B] buffer per output warp (8 x 2 KB)
-  __host__ __device__ static constexpr uint32_t ystage(int w) { return 32768u + (uint32_t)w * 2048u; }
-  static constexpr uint32_t misc = 49152u;  // K3Misc, at most 10 KB
-  static constexpr uint32_t ring = 59392u;  // slot ring; the B rows for G sit at its end until G is formed
+  // y staging: one [32 rows][32 fp32] tile (128-byte swizzle) per output warp, the source
+  // of that warp's TMA store (8 x 4 KB)
+  __host__ __device__ static constexpr uint32_t ystage(int w) { return 32768u + (uint32_t)w * 4096u; }
+  static constexpr uint32_t misc = 65536u;  // K3Misc, at most 10 KB
+  static constexpr uint32_t ring = 75776u;  // slot ring; the B rows for G sit at its end until G is formed
   static constexpr uint32_t end = 231424u;  // 227 KB of dynamic shared memory less the alignment slack
   // slot: nblk x blocks of [128 rows][128 B], then h_prev^T as 2 K-halves of [64][128 B]
   __host__ __device__ static constexpr uint32_t slot_bytes(int nblk) { return (uint32_t)nblk * 16384u + 16384u; }
@@ -389,7 +394,7 @@ struct K3Smem {
   // B rows for G: 2 K-atoms, each [128 * nblk rows][128 B]
   __host__ __device__ static constexpr uint32_t bm(int nblk) { return end - (uint32_t)nblk * 32768u; }
 };
-static_assert(K3Smem::slots(1) == 5 && K3Smem::slots(2) == 3, "slot ring depth");
+static_assert(K3Smem::slots(1) == 4 && K3Smem::slots(2) == 3, "slot ring depth");
 static_assert(K3Smem::ring % 1024 == 0 && K3Smem::bm(1) % 1024 == 0 && K3Smem::bm(2) % 1024 == 0,
               "TMA destinations with 128-byte swizzle must be 1024-byte aligned");
 
@@ -421,9 +426,8 @@ constexpr uint32_t K3_TM_WB = 0, K3_TM_WS = 128, K3_TM_ACC = 256;
 __global__ void __launch_bounds__(K3_THREADS, 1)
 k_chunk_scan_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_C,
                 const __grid_constant__ CUtensorMap tm_B, const __grid_constant__ CUtensorMap tm_h,
-                const __nv_bfloat16 *__restrict__ x, const float *__restrict__ dt, const float *__restrict__ A,
-                const float *__restrict__ D, float *__restrict__ y, int *err,
-                Dims d, int Q, int nc, int kb0, int nhb0, int kb1, int nhb1) {
+                const __grid_constant__ CUtensorMap tm_y, const float *__restrict__ dt, const float *__restrict__ A,
+                const float *__restrict__ D, int *err, Dims d, int Q, int nc, int kb0, int nhb0, int kb1, int nhb1) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   K3Misc *ms = reinterpret_cast<K3Misc *>(base + K3Smem::misc);
@@ -487,6 +491,7 @@ k_chunk_scan_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
       tma_prefetch_desc(&tm_C);
       tma_prefetch_desc(&tm_B);
       tma_prefetch_desc(&tm_h);
+      tma_prefetch_desc(&tm_y);
       const uint32_t bmo = K3Smem::bm(nblk);
       mbar_arrive_expect_tx(&ms->cb_full, 32768u + (uint32_t)nblk * 32768u);
       for (int kn = 0; kn < 2; ++kn)
@@ -569,12 +574,12 @@ k_chunk_scan_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
         }
         if (!mbar_wait(&ms->ops_ready[s], u & 1, abort_flag, err)) break;
         tc_fence_after();
-        // ACC_intra = W X': A from TMEM (W_base, or the head's own W when steep), K = source tokens
+        // ACC_intra += W X': A from TMEM (W_base, or the head's own W when steep), K = source tokens
         const uint32_t wa = tmem + (ms->steep[cb] ? K3_TM_WS : K3_TM_WB);
         for (int jj = 0; jj < nblk; ++jj)
           for (int ks = 0; ks < 8; ++ks) {
             const uint64_t bd = smem_desc_sw128(so + jj * 16384u + ks * 2048u, 16384u, 1024u);
-            mma_bf16_ts(acc + 64, wa + (uint32_t)(64 * jj + 8 * ks), bd, id_intra, (jj > 0 || ks > 0) ? 1u : 0u);
+            mma_bf16_ts(acc + 64, wa + (uint32_t)(64 * jj + 8 * ks), bd, id_intra, 1u);  // onto D x / u
           }
         mma_commit(&ms->acc_full[a]);
         mma_commit(&ms->x_free[s]);
@@ -583,8 +588,8 @@ k_chunk_scan_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
     __syncwarp();
   } else if (warp < 6) {
     // ------------------------------------------------------------- W build and x scaling (128 threads)
-    // Thread (q, lane) owns row tl = 32q + lane of W (TMEM lane tl); the warp's rows are the
-    // 32-token group q of the tile.
+    // Thread (q, lane) owns row tl = 32q + lane of W and of the accumulators (TMEM lane tl);
+    // the warp's rows are the 32-token group q of the tile.
     const int q = warp & 3;
     const int tl = q * 32 + lane;
     const int tid = threadIdx.x - 64;
@@ -621,7 +626,8 @@ k_chunk_scan_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
     named_barrier(1, 128);
     if (tid == 0 && ok) mbar_arrive(&ms->w_ready);
     for (int k = 0; k < nh; ++k) {
-      const int cb = k % K3_CUMBUF, s = k % NS;
+      const int cb = k % K3_CUMBUF, s = k % NS, a = k & 1;
+      const float dh = D[h0 + k];
       ok = ok && mbar_wait(&ms->cum_full[cb], (k / K3_CUMBUF) & 1, abort_flag, err);
       const bool steep = ok && ms->steep[cb];
       if (steep) {
@@ -671,24 +677,59 @@ k_chunk_scan_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
           tmem_st_wait();
         }
       }
-      // scale the rows of this head's x tile by v_s (not for steep heads: their W holds the decay)
+      // Each thread takes row tl of every x block of the slot (the 128-byte swizzle keeps 8
+      // consecutive rows on distinct banks).  In the tile's own block it first stores
+      // D x_t / u_t into the intra accumulator (the MMA adds W X' onto it); then, unless the
+      // head is steep (its W holds the decay), it scales the row by v_s in place.
       ok = ok && mbar_wait(&ms->x_full[s], (k / NS) & 1, abort_flag, err);
-      if (ok && !steep) {
+      if (k >= 2) ok = ok && mbar_wait(&ms->acc_free[a], ((k >> 1) - 1) & 1, abort_flag, err);
+      tc_fence_after();
+      if (ok) {
         const uint32_t xs = smem_u32(base + K3Smem::slot(nblk, s));
-        const float *vt = ms->v[cb];
-        const int units = nblk * 128 * 8;  // 16-byte units: row = unit / 8 (rows of 128 B)
-#pragma unroll 4
-        for (int unit = tid; unit < units; unit += 128) {
-          const float vv = vt[unit >> 3];
-          const uint32_t addr = xs + (uint32_t)unit * 16u;
-          const uint4 in = ld_shared_v4(addr);
-          const uint32_t w4[4] = {in.x, in.y, in.z, in.w};
-          uint32_t o4[4];
+        const float c2t = ms->c2[cb][t];
+        const float dsc = steep ? dh : dh * ex2(ms->c2ref[cb] - c2t);  // D / u_t
+        const uint32_t acc_i = tmem + lane_off + K3_TM_ACC + 128u * a + 64u;
+        for (int jj = 0; jj < nblk; ++jj) {
+          const uint32_t ra = xs + (uint32_t)jj * 16384u + (uint32_t)tl * 128u;
+          const float vv = ms->v[cb][128 * jj + tl];
 #pragma unroll
-          for (int m = 0; m < 4; ++m)
-            o4[m] = pack_bf16x2(__uint_as_float(w4[m] << 16) * vv, __uint_as_float(w4[m] & 0xffff0000u) * vv);
-          st_shared_v4(addr, o4[0], o4[1], o4[2], o4[3]);
+          for (int half = 0; half < 2; ++half) {  // channels 32 half .. 32 half + 31
+            uint32_t w[16];
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc) {
+              const uint4 in = ld_shared_v4(ra + ((uint32_t)((4 * half + cc) ^ (tl & 7)) << 4));
+              w[4 * cc] = in.x;
+              w[4 * cc + 1] = in.y;
+              w[4 * cc + 2] = in.z;
+              w[4 * cc + 3] = in.w;
+            }
+            if (jj == ti) {
+              uint32_t lo[16], hi[16];
+#pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                lo[2 * e] = __float_as_uint(__uint_as_float(w[e] << 16) * dsc);
+                lo[2 * e + 1] = __float_as_uint(__uint_as_float(w[e] & 0xffff0000u) * dsc);
+                hi[2 * e] = __float_as_uint(__uint_as_float(w[8 + e] << 16) * dsc);
+                hi[2 * e + 1] = __float_as_uint(__uint_as_float(w[8 + e] & 0xffff0000u) * dsc);
+              }
+              tmem_st16(acc_i + 32u * half, lo);
+              tmem_st16(acc_i + 32u * half + 16u, hi);
+            }
+            if (!steep) {
+#pragma unroll
+              for (int cc = 0; cc < 4; ++cc) {
+                uint32_t o4[4];
+#pragma unroll
+                for (int m = 0; m < 4; ++m) {
+                  const uint32_t wv = w[4 * cc + m];
+                  o4[m] = pack_bf16x2(__uint_as_float(wv << 16) * vv, __uint_as_float(wv & 0xffff0000u) * vv);
+                }
+                st_shared_v4(ra + ((uint32_t)((4 * half + cc) ^ (tl & 7)) << 4), o4[0], o4[1], o4[2], o4[3]);
+              }
+            }
+          }
         }
+        tmem_st_wait();
       }
       fence_proxy_async_smem();
       tc_fence_before();
@@ -701,93 +742,60 @@ k_chunk_scan_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
   } else if (warp < 14) {
     // ------------------------------------------------------------- output warps (256 threads)
     // Warp (q, hf) owns rows 32q .. 32q + 31 of the tile (TMEM lane quarter q) and the 32
-    // channels [32 hf, 32 hf + 32).  Its 2 KB staging buffer first brings in x (coalesced
-    // row segments) for the D x_t term, then takes y out 16 channels at a time, so every
-    // global access moves whole 64-byte row segments.
+    // channels [32 hf, 32 hf + 32): y_t = e_t ACC_inter + u_t ACC_intra (the latter already
+    // holds D x_t / u_t), written as one swizzled [32][32] fp32 tile and stored by TMA
+    // (rows past the end of the sequence are clipped by the tensor map).
     const int q = warp & 3, hf = (warp - 6) >> 2;
     const int tl = q * 32 + lane;
     const int t = 128 * ti + tl;
     const int tid = threadIdx.x - 192;
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
-    const uint32_t stg = smem_u32(base + K3Smem::ystage(warp - 6));
-    const int row0 = 128 * ti + 32 * q;                  // chunk-relative first row of the warp
-    const int nrows = max(0, min(32, valid - row0));     // rows of this warp that exist
-    // staging layout: 32 rows x 64 bytes, 16-byte chunk c of row r at (c ^ ((r >> 1) & 3))
-    auto sidx = [](int rr, int c) -> uint32_t { return (uint32_t)rr * 64u + ((c ^ ((rr >> 1) & 3)) << 4); };
+    uint8_t *stg = base + K3Smem::ystage(warp - 6);
+    const uint32_t srow = smem_u32(stg) + (uint32_t)lane * 128u;
     for (int k = 0; k < nh; ++k) {
       const int a = k & 1, cb = k % K3_CUMBUF, h = h0 + k;
-      // x rows of this warp (channels of its half), 4 threads per 64-byte row segment
-      const size_t rstride = (size_t)d.H * TP;  // elements between consecutive tokens
-      const __nv_bfloat16 *xw = x + (((size_t)bi * d.L + t0 + row0) * d.H + h) * TP + 32 * hf;
-      uint4 xl[4];
-#pragma unroll
-      for (int it = 0; it < 4; ++it) {
-        const int rr = 8 * it + (lane >> 2), c = lane & 3;
-        xl[it] = (rr < nrows) ? __ldg(reinterpret_cast<const uint4 *>(xw + (size_t)rr * rstride) + c)
-                              : make_uint4(0u, 0u, 0u, 0u);
-      }
       bool ok = mbar_wait(&ms->cum_full[cb], (k / K3_CUMBUF) & 1, abort_flag, err);
       ok = ok && mbar_wait(&ms->acc_full[a], (k >> 1) & 1, abort_flag, err);
       tc_fence_after();
+      float vi[32], va[32];
+      float et = 0.f, ut = 0.f;
       if (ok) {
         const uint32_t acc = tmem + lane_off + K3_TM_ACC + 128u * a + 32u * hf;
-        float vi[32], va[32];
         tmem_ld32(acc, vi);
         tmem_ld32(acc + 64u, va);
-#pragma unroll
-        for (int it = 0; it < 4; ++it) {
-          const int rr = 8 * it + (lane >> 2), c = lane & 3;
-          st_shared_v4(stg + sidx(rr, c), xl[it].x, xl[it].y, xl[it].z, xl[it].w);
-        }
-        __syncwarp();
-        uint32_t xr[16];  // this thread's row: 32 bf16
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const uint4 v4 = ld_shared_v4(stg + sidx(lane, c));
-          xr[4 * c] = v4.x;
-          xr[4 * c + 1] = v4.y;
-          xr[4 * c + 2] = v4.z;
-          xr[4 * c + 3] = v4.w;
-        }
         const float c2t = ms->c2[cb][t];
-        const float et = ex2(c2t);
-        const float ut = ms->steep[cb] ? 1.f : ex2(c2t - ms->c2ref[cb]);
-        const float Dh = D[h];
+        et = ex2(c2t);
+        ut = ms->steep[cb] ? 1.f : ex2(c2t - ms->c2ref[cb]);
         tmem_ld_wait();
-        __syncwarp();
-        float *yw = y + (((size_t)bi * d.L + t0 + row0) * d.H + h) * TP + 32 * hf;
-#pragma unroll
-        for (int pass = 0; pass < 2; ++pass) {  // channels 16 pass .. 16 pass + 15 of the half
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            float o[4];
-#pragma unroll
-            for (int m = 0; m < 4; ++m) {
-              const int e = 16 * pass + 4 * c + m;
-              const uint32_t wv = xr[e >> 1];
-              const float xv = __uint_as_float((e & 1) ? (wv & 0xffff0000u) : (wv << 16));
-              o[m] = fmaf(et, vi[e], fmaf(ut, va[e], Dh * xv));
-            }
-            st_shared_v4(stg + sidx(lane, c), __float_as_uint(o[0]), __float_as_uint(o[1]), __float_as_uint(o[2]),
-                         __float_as_uint(o[3]));
-          }
-          __syncwarp();
-#pragma unroll
-          for (int it = 0; it < 4; ++it) {
-            const int rr = 8 * it + (lane >> 2), c = lane & 3;
-            const uint4 v4 = ld_shared_v4(stg + sidx(rr, c));
-            if (rr < nrows) *reinterpret_cast<uint4 *>(yw + (size_t)rr * rstride + 16 * pass + 4 * c) = v4;
-          }
-          __syncwarp();
-        }
       }
+      // the accumulators and decay tables are read: release them before writing y
       tc_fence_before();
       named_barrier(2, 256);
       if (tid == 0 && ok) {
         mbar_arrive(&ms->acc_free[a]);
         mbar_arrive(&ms->cum_free[cb]);
       }
+      if (ok) {
+        if (lane == 0) tma_store_wait_read();  // the previous head's store has read the tile
+        __syncwarp();
+#pragma unroll
+        for (int cc = 0; cc < 8; ++cc) {
+          float o[4];
+#pragma unroll
+          for (int m = 0; m < 4; ++m) o[m] = fmaf(et, vi[4 * cc + m], ut * va[4 * cc + m]);
+          st_shared_v4(srow + ((uint32_t)(cc ^ (lane & 7)) << 4), __float_as_uint(o[0]), __float_as_uint(o[1]),
+                       __float_as_uint(o[2]), __float_as_uint(o[3]));
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_3d(&tm_y, stg, h * TP + 32 * hf, t0 + 128 * ti + 32 * q, bi);
+          tma_store_commit();
+        }
+      }
     }
+    if (lane == 0) tma_store_wait_all();
+    __syncwarp();
   } else {
     // ------------------------------------------------------------- decay-table warp
     // dt and A of head k + 1 are loaded while head k's buffer is awaited and filled
@@ -1000,12 +1008,13 @@ cudaError_t launch_tc_prefill(const __nv_bfloat16 *x, const float *dt, const flo
                               const __nv_bfloat16 *C, const float *D, float *y, float *final_state, float *states,
                               float *cdecay, __nv_bfloat16 *hprev, int *err, const Dims &d, int Q, int nc,
                               cudaStream_t st, const cudaEvent_t *ev) {
-  CUtensorMap tm_x1, tm_B1, tm_x3, tm_C3, tm_B3, tm_h3;
+  CUtensorMap tm_x1, tm_B1, tm_x3, tm_C3, tm_B3, tm_h3, tm_y3;
   const uint64_t HP = (uint64_t)d.H * d.P, GN = (uint64_t)d.G * d.N;
   if (!make_map(&tm_x1, x, HP, d.L, d.b, Q) || !make_map(&tm_B1, B, GN, d.L, d.b, Q) ||
       !make_map(&tm_x3, x, HP, d.L, d.b, 128) || !make_map(&tm_C3, C, GN, d.L, d.b, 128) ||
       !make_map(&tm_B3, B, GN, d.L, d.b, 128) ||
-      !make_map(&tm_h3, hprev, (uint64_t)d.N, (uint64_t)d.P, (uint64_t)d.b * nc * d.H, 64))
+      !make_map(&tm_h3, hprev, (uint64_t)d.N, (uint64_t)d.P, (uint64_t)d.b * nc * d.H, 64) ||
+      !make_map_t(&tm_y3, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, y, HP, d.L, d.b, 32, 32))
     return cudaErrorInvalidValue;
   const int sms = num_sms();
   auto mark = [&](int i) { return ev ? cudaEventRecord(ev[i], st) : cudaSuccess; };
@@ -1043,7 +1052,7 @@ cudaError_t launch_tc_prefill(const __nv_bfloat16 *x, const float *dt, const flo
     e = cudaFuncSetAttribute(k_chunk_scan_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kK3SmemBytes);
     if (e != cudaSuccess) return e;
     e = launch_after(dim3((unsigned)(groups * (sp.nhb0 + sp.nhb1))), K3_THREADS, kK3SmemBytes, st, pdl,
-                     k_chunk_scan_tc, tm_x3, tm_C3, tm_B3, tm_h3, x, dt, A, D, y, err, d, Q, nc, sp.kb0, sp.nhb0,
+                     k_chunk_scan_tc, tm_x3, tm_C3, tm_B3, tm_h3, tm_y3, dt, A, D, err, d, Q, nc, sp.kb0, sp.nhb0,
                      sp.kb1, sp.nhb1);
     if (e != cudaSuccess) return e;
   }
