@@ -371,7 +371,8 @@ k_state_passing_bf16(const float *__restrict__ states, const float *__restrict__
 // x row anyway, store D x_t / u_t into the intra-chunk accumulator before the MMA adds
 // W X' onto it; the output warps then only combine the two accumulators and hand each
 // [32 rows][32 channels] tile of y to a TMA store.
-constexpr int K3_THREADS = 480;  // warp 0 TMA, 1 MMA, 2-5 W/x scaling, 6-13 output, 14 decay tables
+constexpr int K3_THREADS = 512;  // warp 0 TMA, 1 MMA (G, inter), 2-5 W/x scaling, 6-13 output, 14 decay
+                                 // tables, 15 MMA (intra)
 constexpr int K3_CUMBUF = 3;
 constexpr int K3_MAXSLOTS = 5;
 constexpr float kSteepLog2 = 100.f;
@@ -461,10 +462,10 @@ k_chunk_scan_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
     for (int s = 0; s < K3_MAXSLOTS; ++s) {
       mbar_init(&ms->x_full[s], 1);
       mbar_init(&ms->ops_ready[s], 1);
-      mbar_init(&ms->x_free[s], 1);  // MMA commit
+      mbar_init(&ms->x_free[s], 2);  // commits of both MMA issuers
     }
     for (int a = 0; a < 2; ++a) {
-      mbar_init(&ms->acc_full[a], 1);
+      mbar_init(&ms->acc_full[a], 2);  // commits of both MMA issuers
       mbar_init(&ms->acc_free[a], 1);
     }
     for (int s = 0; s < K3_CUMBUF; ++s) {
@@ -539,7 +540,10 @@ k_chunk_scan_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
     }
     __syncwarp();
   } else if (warp == 1) {
-    // ------------------------------------------------------------- MMA issuer
+    // ------------------------------------------------------------- MMA issuer: G, then ACC_inter
+    // A single thread issues one tcgen05.mma about every 65 ns whatever N is up to 128, so
+    // the inter-chunk and intra-chunk products are issued by two warps (this one and warp 15)
+    // into their own accumulators; each commits to acc_full and x_free (count 2).
     if (lane == 0) {
       const uint32_t cm = smem_u32(base + K3Smem::cm), bmm = smem_u32(base + K3Smem::bm(nblk));
       bool ok = mbar_wait(&ms->cb_full, 0, abort_flag, err);
@@ -557,9 +561,8 @@ k_chunk_scan_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
       // G occupies the accumulator columns until W_base has been built from it
       ok = ok && mbar_wait(&ms->w_ready, 0, abort_flag, err);
       const uint32_t id_inter = idesc_bf16_f32(128, TP, false, false);
-      const uint32_t id_intra = idesc_bf16_f32(128, TP, false, true);
       for (int k = 0; ok && k < nh; ++k) {
-        const int s = k % NS, u = k / NS, a = k & 1, cb = k % K3_CUMBUF;
+        const int s = k % NS, u = k / NS, a = k & 1;
         if (!mbar_wait(&ms->x_full[s], u & 1, abort_flag, err)) break;
         if (k >= 2 && !mbar_wait(&ms->acc_free[a], ((k >> 1) - 1) & 1, abort_flag, err)) break;
         tc_fence_after();
@@ -572,15 +575,6 @@ k_chunk_scan_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
           const uint64_t bd = smem_desc_sw128(hsa + (ks >> 2) * 8192u + (ks & 3) * 32u, 16u, 1024u);
           mma_bf16(acc, ad, bd, id_inter, ks > 0 ? 1u : 0u);
         }
-        if (!mbar_wait(&ms->ops_ready[s], u & 1, abort_flag, err)) break;
-        tc_fence_after();
-        // ACC_intra += W X': A from TMEM (W_base, or the head's own W when steep), K = source tokens
-        const uint32_t wa = tmem + (ms->steep[cb] ? K3_TM_WS : K3_TM_WB);
-        for (int jj = 0; jj < nblk; ++jj)
-          for (int ks = 0; ks < 8; ++ks) {
-            const uint64_t bd = smem_desc_sw128(so + jj * 16384u + ks * 2048u, 16384u, 1024u);
-            mma_bf16_ts(acc + 64, wa + (uint32_t)(64 * jj + 8 * ks), bd, id_intra, 1u);  // onto D x / u
-          }
         mma_commit(&ms->acc_full[a]);
         mma_commit(&ms->x_free[s]);
       }
@@ -795,6 +789,30 @@ k_chunk_scan_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
       }
     }
     if (lane == 0) tma_store_wait_all();
+    __syncwarp();
+  } else if (warp == 15) {
+    // ------------------------------------------------------------- MMA issuer: ACC_intra
+    // ops_ready implies x_full, acc_free and W_base: the scaling warps waited for all three
+    // before storing D x / u into the accumulator this MMA adds onto.
+    if (lane == 0) {
+      const uint32_t id_intra = idesc_bf16_f32(128, TP, false, true);
+      for (int k = 0; k < nh; ++k) {
+        const int s = k % NS, u = k / NS, a = k & 1, cb = k % K3_CUMBUF;
+        if (!mbar_wait(&ms->ops_ready[s], u & 1, abort_flag, err)) break;
+        tc_fence_after();
+        const uint32_t acc = tmem + K3_TM_ACC + 128u * a;
+        const uint32_t so = smem_u32(base + K3Smem::slot(nblk, s));
+        // ACC_intra += W X': A from TMEM (W_base, or the head's own W when steep), K = source tokens
+        const uint32_t wa = tmem + (ms->steep[cb] ? K3_TM_WS : K3_TM_WB);
+        for (int jj = 0; jj < nblk; ++jj)
+          for (int ks = 0; ks < 8; ++ks) {
+            const uint64_t bd = smem_desc_sw128(so + jj * 16384u + ks * 2048u, 16384u, 1024u);
+            mma_bf16_ts(acc + 64, wa + (uint32_t)(64 * jj + 8 * ks), bd, id_intra, 1u);  // onto D x / u
+          }
+        mma_commit(&ms->acc_full[a]);
+        mma_commit(&ms->x_free[s]);
+      }
+    }
     __syncwarp();
   } else {
     // ------------------------------------------------------------- decay-table warp
