@@ -64,21 +64,23 @@ constexpr int TP = 64;    // headdim handled by the tensor-core path
 constexpr int TN = 128;   // d_state handled by the tensor-core path
 
 // ============================================================================ K1
-constexpr int K1_SLOTS = 2;
+constexpr int K1_SLOTS = 3;
 constexpr int K1_CUMBUF = 3;
 constexpr int K1_THREADS = 480;  // warp 0 TMA, 1 MMA, 2-9 scale, 10-13 epilogue, 14 decay weights
 
 struct K1Smem {
   // offsets from the 1024-aligned base
-  static constexpr uint32_t bm = 0;  // B chunk: 2 x [Q][128 B]
   // slot s: x (scaled in place to the bf16 high part), directly followed by its remainder
-  __host__ __device__ static constexpr uint32_t x(int Q, int s) { return 2u * Q * 128u + (uint32_t)s * 2u * Q * 128u; }
+  __host__ __device__ static constexpr uint32_t x(int Q, int s) { return (uint32_t)s * 2u * Q * 128u; }
   __host__ __device__ static constexpr uint32_t lo(int Q, int s) { return x(Q, s) + (uint32_t)Q * 128u; }
-  __host__ __device__ static constexpr uint32_t misc(int Q) { return 2u * Q * 128u + K1_SLOTS * 2u * Q * 128u; }
+  // the B chunk (2 x [Q][128 B]) lands in the last slot and is moved to TMEM before that
+  // slot's first use
+  __host__ __device__ static constexpr uint32_t bm(int Q) { return x(Q, K1_SLOTS - 1); }
+  __host__ __device__ static constexpr uint32_t misc(int Q) { return K1_SLOTS * 2u * Q * 128u; }
 };
 
 struct K1Misc {
-  uint64_t b_full;
+  uint64_t b_full, b_tmem;
   uint64_t x_full[K1_SLOTS], scaled[K1_SLOTS], x_free[K1_SLOTS];
   uint64_t acc_full[2], acc_free[2];
   uint64_t w_full[K1_CUMBUF], w_free[K1_CUMBUF];
@@ -86,6 +88,9 @@ struct K1Misc {
   int abort_flag;
   float w[K1_CUMBUF][256];  // decay weights exp(cum_end - cum_t) dt_t of upcoming heads
 };
+
+// TMEM columns: two accumulator slots of [high 64 | remainder 64], then B chunk^T (Q / 2).
+constexpr uint32_t K1_TM_B = 256, K1_TM_COLS = 512;  // allocation: a power of two >= 256 + Q / 2
 
 __global__ void __launch_bounds__(K1_THREADS, 1)
 k_chunk_state_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_B,
@@ -112,6 +117,7 @@ k_chunk_state_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
 
   if (threadIdx.x == 0) {
     mbar_init(&ms->b_full, 1);
+    mbar_init(&ms->b_tmem, 1);
     for (int s = 0; s < K1_SLOTS; ++s) {
       mbar_init(&ms->x_full[s], 1);
       mbar_init(&ms->scaled[s], 1);
@@ -129,7 +135,7 @@ k_chunk_state_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
     mbar_fence_init();
   }
   if (warp == 1) {
-    tmem_alloc(&ms->tmem, 256);
+    tmem_alloc(&ms->tmem, K1_TM_COLS);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -144,12 +150,14 @@ k_chunk_state_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
       tma_prefetch_desc(&tm_x);
       tma_prefetch_desc(&tm_B);
       mbar_arrive_expect_tx(&ms->b_full, 2u * Q * 128u);
-      tma_load_3d(base + K1Smem::bm, &tm_B, &ms->b_full, g * TN, t0, bi);
-      tma_load_3d(base + K1Smem::bm + (uint32_t)Q * 128u, &tm_B, &ms->b_full, g * TN + 64, t0, bi);
+      tma_load_3d(base + K1Smem::bm(Q), &tm_B, &ms->b_full, g * TN, t0, bi);
+      tma_load_3d(base + K1Smem::bm(Q) + (uint32_t)Q * 128u, &tm_B, &ms->b_full, g * TN + 64, t0, bi);
       int issued = 0;
       for (int k = 0; k < nh; ++k) {
         const int s = k % K1_SLOTS, u = k / K1_SLOTS;
         if (k >= K1_SLOTS && !mbar_wait(&ms->x_free[s], (u - 1) & 1, abort_flag, err)) break;
+        // the last slot holds the B chunk until it has been moved to TMEM
+        if (k == K1_SLOTS - 1 && !mbar_wait(&ms->b_tmem, 0, abort_flag, err)) break;
         mbar_arrive_expect_tx(&ms->x_full[s], (uint32_t)Q * 128u);
         tma_load_3d(base + K1Smem::x(Q, s), &tm_x, &ms->x_full[s], (h0 + k) * TP, t0, bi);
         issued = k + 1;
@@ -164,9 +172,9 @@ k_chunk_state_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
   } else if (warp == 1) {
     // ------------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      const uint32_t idesc = idesc_bf16_f32(128, 2 * TP, /*a MN-major*/ true, /*b MN-major*/ true);
-      const uint32_t bm_addr = smem_u32(base + K1Smem::bm);
-      bool ok = mbar_wait(&ms->b_full, 0, abort_flag, err);
+      // A = B chunk^T from TMEM: [M = d_state lanes][K = token], bf16 pairs along K
+      const uint32_t idesc = idesc_bf16_f32(128, 2 * TP, /*a MN-major*/ false, /*b MN-major*/ true);
+      bool ok = mbar_wait(&ms->b_tmem, 0, abort_flag, err);
       for (int k = 0; ok && k < nh; ++k) {
         const int s = k % K1_SLOTS, a = k & 1;
         if (!mbar_wait(&ms->scaled[s], (k / K1_SLOTS) & 1, abort_flag, err)) break;
@@ -174,11 +182,9 @@ k_chunk_state_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
         tc_fence_after();
         const uint32_t x_addr = smem_u32(base + K1Smem::x(Q, s));
         for (int ks = 0; ks < Q / 16; ++ks) {
-          // A = B chunk as [M = d_state][K = token], d_state contiguous (two 64-wide blocks Q*128 B apart)
-          const uint64_t ad = smem_desc_sw128(bm_addr + ks * 2048u, (uint32_t)Q * 128u, 1024u);
           // B = [K = token][N = (high | remainder) x channel]: two 64-wide blocks Q*128 B apart
           const uint64_t bd = smem_desc_sw128(x_addr + ks * 2048u, (uint32_t)Q * 128u, 1024u);
-          mma_bf16(tmem + (uint32_t)(a * 2 * TP), ad, bd, idesc, ks > 0 ? 1u : 0u);
+          mma_bf16_ts(tmem + (uint32_t)(a * 2 * TP), tmem + K1_TM_B + 8u * ks, bd, idesc, ks > 0 ? 1u : 0u);
         }
         mma_commit(&ms->acc_full[a]);
         mma_commit(&ms->x_free[s]);
@@ -227,6 +233,34 @@ k_chunk_state_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
     const int q = warp & 3;
     const int n = q * 32 + lane;  // d_state row of the accumulator
     const int tid = threadIdx.x - 320;
+    {
+      // First move the B chunk into TMEM as the MMA's A operand: lane n gets B[t][n] for
+      // every token, packed in pairs (t even in the low half).  In shared memory (128-byte
+      // swizzle) 16-byte chunk j of row t of a 64-wide block sits at chunk j ^ (t & 7).
+      bool ok = mbar_wait(&ms->b_full, 0, abort_flag, err);
+      if (ok) {
+        const uint32_t src = smem_u32(base + K1Smem::bm(Q)) + (uint32_t)(n >> 6) * (uint32_t)Q * 128u +
+                             (uint32_t)(n & 7) * 2u;
+        const uint32_t j8 = (uint32_t)((n & 63) >> 3);
+        const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+        for (int c0 = 0; c0 < Q / 2; c0 += 16) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const uint32_t t = 2u * (uint32_t)(c0 + e);
+            const uint32_t b0 = ld_shared_u16(src + t * 128u + ((j8 ^ (t & 7u)) << 4));
+            const uint32_t b1 = ld_shared_u16(src + (t + 1u) * 128u + ((j8 ^ ((t + 1u) & 7u)) << 4));
+            pk[e] = b0 | (b1 << 16);
+          }
+          tmem_st16(tmem + lane_off + K1_TM_B + (uint32_t)c0, pk);
+        }
+        tmem_st_wait();
+      }
+      fence_proxy_async_smem();  // the slot is refilled by TMA after these reads
+      tc_fence_before();
+      named_barrier(2, 128);
+      if (tid == 0 && ok) mbar_arrive(&ms->b_tmem);
+    }
     for (int k = 0; k < nh; ++k) {
       const int a = k & 1, h = h0 + k;
       const bool ok = mbar_wait(&ms->acc_full[a], (k >> 1) & 1, abort_flag, err);
@@ -300,7 +334,7 @@ k_chunk_state_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 256);
+    tmem_dealloc(tmem, K1_TM_COLS);
   }
 }
 
