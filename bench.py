@@ -225,6 +225,7 @@ def kernel_work(name, w, Q):
     el = 2 if w.dtype == "bf16" else 4
     x_b, bc_b, dt_b = tok * H * P * el, tok * G * N * el, tok * H * 4
     states = b * nc * H * P * N
+    tab_b = b * H * nc * (4 + 2 * Q) * 4   # decay table rows (tensor-core path)
     flops_state = tok * H * 2 * N * P
     flops_scan = tok * H * (2 * Q * P + 2 * N * P) + tok * G * 2 * Q * N
     if name.startswith("dA_cumsum"):
@@ -234,9 +235,9 @@ def kernel_work(name, w, Q):
     if name.startswith("state_passing"):
         return "hbm", states * 4 + states * 2 + b * H * P * N * 4 + b * H * nc * 4, "bytes", 0
     if name == "chunk_state_tc":
-        return "hbm", x_b + bc_b + dt_b + states * 4 + b * H * nc * 4, "bytes", flops_state
+        return "hbm", x_b + bc_b + dt_b + tab_b + states * 4 + b * H * nc * 4, "bytes", flops_state
     if name == "chunk_scan_tc":
-        return "hbm", x_b + 2 * bc_b + dt_b + states * 2 + tok * H * P * 4, "bytes", flops_scan
+        return "hbm", x_b + 2 * bc_b + tab_b + states * 2 + tok * H * P * 4, "bytes", flops_scan
     if name.startswith("chunk_state"):
         return "flops", flops_state, "flops", flops_state
     if name.startswith("chunk_scan"):

@@ -25,10 +25,12 @@ size_t chunk_scan_simt_smem_bytes(int N);
 
 // prefill_tc.cu (bf16 x/B/C, P = 64, N = 128, Q in {128, 256})
 bool tc_prefill_supported(const Dims &d, int Q);
+// floats of the per-(batch, head, chunk) decay table the tensor-core kernels share
+size_t tc_prefill_table_floats(const Dims &d, int Q, int nc);
 cudaError_t launch_tc_prefill(const __nv_bfloat16 *x, const float *dt, const float *A, const __nv_bfloat16 *B,
-                              const __nv_bfloat16 *C, const float *D, float *y, float *final_state, float *states,
-                              float *cdecay, __nv_bfloat16 *hprev, int *err, const Dims &d, int Q, int nc,
-                              cudaStream_t st, const cudaEvent_t *ev);
+                              const __nv_bfloat16 *C, const float *D, float *y, float *final_state, float *tab,
+                              float *states, float *cdecay, __nv_bfloat16 *hprev, int *err, const Dims &d, int Q,
+                              int nc, cudaStream_t st, const cudaEvent_t *ev);
 
 // decode.cu
 template <typename T>

@@ -6,24 +6,29 @@
 // Three kernels:
 //
 //  K1 k_chunk_state_tc   S_c^T[n, p] = sum_t B_t[n] * (exp(cum_end - cum_t) dt_t x_t[p])
-//                        One CTA per (batch, chunk, group, block of heads).  TMA brings
-//                        B_c (once) and each head's x tile (ring of 2 slots); eight warps
-//                        scale x's rows by the decay weight in fp32 and split the product
-//                        into a bf16 high part and a bf16 remainder, stored side by side;
-//                        one thread issues tcgen05.mma with both as the two 64-wide halves
-//                        of N = 128 (M = 128 d_state rows, K = Q tokens), and four warps
-//                        add the halves and stream S_c out in fp32, so the state is
-//                        accurate to fp32 level rather than bf16 level.  Also writes the
-//                        chunk's total decay exp(cum_end).
+//                        One CTA per (batch, chunk, group, block of heads).  While TMA
+//                        brings B_c (once) and the first x tiles, the scale warps form the
+//                        per-chunk dt.A cumulative sums of the CTA's heads: the in-chunk
+//                        cumulative log2-decay c2_t = log2(e) A_h sum_{s<=t} dt_s and dt,
+//                        kept in shared memory and written out head-major as one table row
+//                        per (batch, head, chunk) for the chunk-scan kernel, plus the
+//                        chunk's total decay 2^c2_end for state passing.  Then, per head
+//                        (ring of 3 x slots), eight warps scale x's rows by the decay weight in fp32 and
+//                        split the product into a bf16 high part and a bf16 remainder,
+//                        stored side by side; one thread issues tcgen05.mma with both as
+//                        the two 64-wide halves of N = 128 (M = 128 d_state rows, K = Q
+//                        tokens), and four warps add the halves and stream S_c out in
+//                        fp32, so the state is accurate to fp32 level rather than bf16.
 //  K2 k_state_passing_bf16
 //                        h_c = exp(cum_end,c) h_{c-1} + S_c over chunks in fp32 (the
 //                        first-order recurrence of "Mamba and Selective State Space
 //                        Models" section 5); writes the state entering each chunk in bf16
 //                        (the next kernel's MMA operand) and the final state in fp32.
 //  K3 k_chunk_scan_tc    One CTA per (batch, chunk, 128-row token tile, group, block of
-//                        heads).  G = C_tile B_chunk^T is computed once into TMEM and,
-//                        masked, converted once to a head-independent bf16 W (see the
-//                        decay factorisation at K3 below); per head, 4 warps scale the
+//                        heads), decay data from K1's table.  G = C_tile B_chunk^T is
+//                        computed once into TMEM and, masked, converted once to a
+//                        head-independent bf16 W (see the decay factorisation at K3
+//                        below); per head, 4 warps scale the
 //                        rows of its x tile by the column decay factors, tcgen05.mma forms
 //                        ACC_inter = C_tile h_prev^T and ACC_intra = W X' (double-buffered
 //                        in TMEM across heads), and 8 warps write
@@ -63,10 +68,17 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr int TP = 64;    // headdim handled by the tensor-core path
 constexpr int TN = 128;   // d_state handled by the tensor-core path
 
+// ============================================================================ decay table
+// Decay table row of one (batch, head, chunk), floats, 16-byte aligned:
+//   [0] D_h, [1] 2^c2_end (the chunk's total decay), [2] c2_end, [3] 0,
+//   [4 .. 4+Q) c2_t, the in-chunk cumulative log2-decay through token t,
+//   [4+Q .. 4+2Q) dt_t (0 past the end of the sequence, so c2 stays flat there).
+__host__ __device__ constexpr int tab_row_floats(int Q) { return 4 + 2 * Q; }
+constexpr int kTabHdr = 4;
 // ============================================================================ K1
 constexpr int K1_SLOTS = 3;
-constexpr int K1_CUMBUF = 3;
-constexpr int K1_THREADS = 480;  // warp 0 TMA, 1 MMA, 2-9 scale, 10-13 epilogue, 14 decay weights
+constexpr int K1_THREADS = 448;  // warp 0 TMA, 1 MMA, 2-9 scale (and decay tables), 10-13 epilogue
+constexpr int K1_KB_MAX = 10;    // heads per CTA at most (their decay tables stay in shared memory)
 
 struct K1Smem {
   // offsets from the 1024-aligned base
@@ -83,19 +95,20 @@ struct K1Misc {
   uint64_t b_full, b_tmem;
   uint64_t x_full[K1_SLOTS], scaled[K1_SLOTS], x_free[K1_SLOTS];
   uint64_t acc_full[2], acc_free[2];
-  uint64_t w_full[K1_CUMBUF], w_free[K1_CUMBUF];
   uint32_t tmem;
   int abort_flag;
-  float w[K1_CUMBUF][256];  // decay weights exp(cum_end - cum_t) dt_t of upcoming heads
+  alignas(16) float tab[K1_KB_MAX][tab_row_floats(256)];  // decay table rows of the CTA's heads
 };
+static_assert(offsetof(K1Misc, tab) % 16 == 0, "bulk-copy destinations must be 16-byte aligned");
 
 // TMEM columns: two accumulator slots of [high 64 | remainder 64], then B chunk^T (Q / 2).
 constexpr uint32_t K1_TM_B = 256, K1_TM_COLS = 512;  // allocation: a power of two >= 256 + Q / 2
 
 __global__ void __launch_bounds__(K1_THREADS, 1)
 k_chunk_state_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_B,
-                 const float *__restrict__ dt, const float *__restrict__ A, float *__restrict__ states,
-                 float *__restrict__ cdecay, int *err, Dims d, int Q, int nc, int kb, int nhb) {
+                 const float *__restrict__ dt, const float *__restrict__ A, const float *__restrict__ D,
+                 float *__restrict__ tab, float *__restrict__ cdecay, float *__restrict__ states, int *err, Dims d, int Q,
+                 int nc, int kb, int nhb) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   K1Misc *ms = reinterpret_cast<K1Misc *>(base + K1Smem::misc(Q));
@@ -126,10 +139,6 @@ k_chunk_state_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
     for (int a = 0; a < 2; ++a) {
       mbar_init(&ms->acc_full[a], 1);
       mbar_init(&ms->acc_free[a], 1);
-    }
-    for (int i = 0; i < K1_CUMBUF; ++i) {
-      mbar_init(&ms->w_full[i], 1);
-      mbar_init(&ms->w_free[i], 1);
     }
     ms->abort_flag = 0;
     mbar_fence_init();
@@ -193,18 +202,78 @@ k_chunk_state_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
     __syncwarp();
   } else if (warp < 10) {
     // ------------------------------------------------------------- scale warps (256 threads)
-    const int tid = threadIdx.x - 64;
+    const int tid = threadIdx.x - 64, wl = warp - 2;
+    {
+      // Decay tables first (per-chunk dt.A cumulative sums), one head per warp and round:
+      // every lane sums Q/32 consecutive tokens, a shuffle scan adds the lanes' totals.
+      // All loads of both rounds are issued before the first use.
+      const int per = Q / 32;
+      float dv[2][8], av[2] = {0.f, 0.f}, dd[2] = {0.f, 0.f};
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        const int k = wl + 8 * r, h = h0 + k;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int t = lane * per + j;
+          dv[r][j] = (k < nh && j < per && t < valid) ? __ldg(dt + ((size_t)bi * d.L + t0 + t) * d.H + h) : 0.f;
+        }
+        if (k < nh) {
+          av[r] = __ldg(A + h);
+          dd[r] = __ldg(D + h);
+        }
+      }
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        const int k = wl + 8 * r, h = h0 + k;
+        if (k >= nh) break;
+        const float a2 = av[r] * kLog2e;
+        float c2v[8];
+        float run = 0.f;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          run += dv[r][j] * a2;
+          c2v[j] = run;
+        }
+        float incl = run;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const float u = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += u;
+        }
+        const float excl = incl - run;
+        const float cend = __shfl_sync(0xffffffffu, incl, 31);
+        float *row = ms->tab[k];
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          if (j < per) {
+            row[kTabHdr + lane * per + j] = c2v[j] + excl;
+            row[kTabHdr + Q + lane * per + j] = dv[r][j];
+          }
+        if (lane == 0) {
+          const float dec = ex2(cend);
+          *reinterpret_cast<float4 *>(row) = make_float4(dd[r], dec, cend, 0.f);
+          cdecay[((size_t)bi * d.H + h) * nc + c] = dec;
+        }
+        __syncwarp();
+        // the row, coalesced, for the chunk-scan kernel
+        float4 *dst = reinterpret_cast<float4 *>(tab + (((size_t)bi * d.H + h) * nc + c) * (size_t)tab_row_floats(Q));
+        for (int j = lane; j < tab_row_floats(Q) / 4; j += 32) dst[j] = reinterpret_cast<const float4 *>(row)[j];
+      }
+      named_barrier(1, 256);  // every head's table row is in shared memory
+    }
+    // Row t of a slot is scaled by w_t = 2^(c2_end - c2_t) dt_t from its head's table row.
     for (int k = 0; k < nh; ++k) {
-      const int s = k % K1_SLOTS, wb = k % K1_CUMBUF;
-      bool ok = mbar_wait(&ms->w_full[wb], (k / K1_CUMBUF) & 1, abort_flag, err);
-      ok = ok && mbar_wait(&ms->x_full[s], (k / K1_SLOTS) & 1, abort_flag, err);
+      const int s = k % K1_SLOTS;
+      const bool ok = mbar_wait(&ms->x_full[s], (k / K1_SLOTS) & 1, abort_flag, err);
       if (ok) {
         const uint32_t xs = smem_u32(base + K1Smem::x(Q, s));
         const uint32_t ls = smem_u32(base + K1Smem::lo(Q, s));
-        const float *wv_row = ms->w[wb];
+        const float *tr = ms->tab[k];
+        const float cend = tr[2];
 #pragma unroll 4
         for (int unit = tid; unit < Q * 8; unit += 256) {
-          const float wv = wv_row[unit >> 3];
+          const int t = unit >> 3;
+          const float wv = ex2(cend - tr[kTabHdr + t]) * tr[kTabHdr + Q + t];
           const uint32_t off = (uint32_t)unit * 16u;  // rows are 128 B: unit*16 = row*128 + chunk*16
           const uint4 v = ld_shared_v4(xs + off);
           const uint32_t in[4] = {v.x, v.y, v.z, v.w};
@@ -214,8 +283,8 @@ k_chunk_state_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
             const float a0 = __uint_as_float(in[q] << 16) * wv;  // exact x * w in fp32
             const float a1 = __uint_as_float(in[q] & 0xffff0000u) * wv;
             hi[q] = pack_bf16x2(a0, a1);
-            const float h0 = __uint_as_float(hi[q] << 16), h1 = __uint_as_float(hi[q] & 0xffff0000u);
-            rem[q] = pack_bf16x2(a0 - h0, a1 - h1);
+            const float h0f = __uint_as_float(hi[q] << 16), h1f = __uint_as_float(hi[q] & 0xffff0000u);
+            rem[q] = pack_bf16x2(a0 - h0f, a1 - h1f);
           }
           st_shared_v4(xs + off, hi[0], hi[1], hi[2], hi[3]);
           st_shared_v4(ls + off, rem[0], rem[1], rem[2], rem[3]);
@@ -223,12 +292,9 @@ k_chunk_state_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
       }
       fence_proxy_async_smem();
       named_barrier(1, 256);
-      if (tid == 0 && ok) {
-        mbar_arrive(&ms->scaled[s]);
-        mbar_arrive(&ms->w_free[wb]);
-      }
+      if (tid == 0 && ok) mbar_arrive(&ms->scaled[s]);
     }
-  } else if (warp < 14) {
+  } else {
     // ------------------------------------------------------------- epilogue warps (128 threads)
     const int q = warp & 3;
     const int n = q * 32 + lane;  // d_state row of the accumulator
@@ -280,53 +346,6 @@ k_chunk_state_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
       tc_fence_before();
       named_barrier(2, 128);
       if (tid == 0) mbar_arrive(&ms->acc_free[a]);
-    }
-  } else {
-    // ------------------------------------------------------------- decay-weight warp
-    // w_t = exp(cum_end - cum_t) dt_t for each upcoming head (ring of K1_CUMBUF), and the
-    // chunk's total decay exp(cum_end) for the state-passing kernel.
-    // dt and A of head k + 1 are loaded while head k's buffer is awaited and filled
-    const int per = Q / 32;
-    auto load_head = [&](int k, float (&v)[8], float &a) {
-      const int h = h0 + k;
-      a = A[h];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int t = lane * per + j;
-        v[j] = (j < per && t < valid) ? dt[((size_t)bi * d.L + t0 + t) * d.H + h] : 0.f;
-      }
-    };
-    float dtv[8], dtn[8], acur = 0.f, anxt = 0.f;
-    if (nh > 0) load_head(0, dtv, acur);
-    for (int k = 0; k < nh; ++k) {
-      const int wb = k % K1_CUMBUF, h = h0 + k;
-      if (k + 1 < nh) load_head(k + 1, dtn, anxt);
-      if (k >= K1_CUMBUF && !mbar_wait(&ms->w_free[wb], ((k / K1_CUMBUF) - 1) & 1, abort_flag, err)) break;
-      const float a2 = acur * kLog2e;
-      float c2[8];
-      float run = 0.f;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        run += dtv[j] * a2;
-        c2[j] = run;
-      }
-      float incl = run;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const float v = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += v;
-      }
-      const float excl = incl - run;
-      const float cend = __shfl_sync(0xffffffffu, incl, 31);
-#pragma unroll
-      for (int j = 0; j < 8; ++j)
-        if (j < per) ms->w[wb][lane * per + j] = ex2(cend - (c2[j] + excl)) * dtv[j];
-      if (lane == 0) cdecay[((size_t)bi * d.H + h) * nc + c] = ex2(cend);
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&ms->w_full[wb]);
-#pragma unroll
-      for (int j = 0; j < 8; ++j) dtv[j] = dtn[j];
-      acur = anxt;
     }
   }
 
@@ -405,9 +424,9 @@ k_state_passing_bf16(const float *__restrict__ states, const float *__restrict__
 // x row anyway, store D x_t / u_t into the intra-chunk accumulator before the MMA adds
 // W X' onto it; the output warps then only combine the two accumulators and hand each
 // [32 rows][32 channels] tile of y to a TMA store.
-constexpr int K3_THREADS = 512;  // warp 0 TMA, 1 MMA (G, inter), 2-5 W/x scaling, 6-13 output, 14 decay
-                                 // tables, 15 MMA (intra)
-constexpr int K3_CUMBUF = 3;
+constexpr int K3_THREADS = 544;  // warp 0 TMA, 1 MMA (G, inter), 2-5 W/x scaling, 6-13 output, 14 decay-table
+                                 // loads, 15 MMA (intra, source block 0), 16 MMA (intra, source block 1)
+constexpr int K3_CUMBUF = 4;
 constexpr int K3_MAXSLOTS = 5;
 constexpr float kSteepLog2 = 100.f;
 
@@ -437,32 +456,53 @@ struct K3Misc {
   uint64_t cb_full, g_full, w_ready;
   uint64_t x_full[K3_MAXSLOTS], ops_ready[K3_MAXSLOTS], x_free[K3_MAXSLOTS];
   uint64_t acc_full[2], acc_free[2];
-  uint64_t cum_full[K3_CUMBUF], cum_free[K3_CUMBUF];
+  uint64_t tab_full[K3_CUMBUF], cum_free[K3_CUMBUF];
   uint32_t tmem;
   int abort_flag;
-  int steep[K3_CUMBUF];
-  float c2ref[K3_CUMBUF];
-  // tables are read with 16-byte vector loads: keep every row 16-byte aligned
-  alignas(16) float c2[K3_CUMBUF][256];   // in-chunk cumulative log2-decay
-  alignas(16) float dts[K3_CUMBUF][256];  // dt of each token of the chunk (0 past the end)
-  alignas(16) float v[K3_CUMBUF][256];    // 2^(c2_r - c2_s) dt_s, s < 128 * (ti + 1)
+  alignas(16) float tab[K3_CUMBUF][tab_row_floats(256)];  // decay table rows of upcoming heads (bulk copies)
 };
-static_assert(offsetof(K3Misc, c2) % 16 == 0 && offsetof(K3Misc, v) % 16 == 0, "decay tables must be 16-byte aligned");
+static_assert(offsetof(K3Misc, tab) % 16 == 0, "bulk-copy destinations must be 16-byte aligned");
 static_assert(K3Smem::misc % 16 == 0, "K3Misc must start 16-byte aligned");
 static_assert(K3Smem::misc + sizeof(K3Misc) <= K3Smem::ring, "K3Misc overlaps the slot ring");
 
 constexpr size_t kK3SmemBytes = 1024 + K3Smem::end;
 
-// TMEM columns: W_base and a steep head's W (bf16 pairs, 64 columns per 128-token block),
-// then two accumulator slots of [inter 64 | intra 64] columns.  G (fp32, 128 * nblk
-// columns) occupies the accumulator slots until W_base has been built from it.
-constexpr uint32_t K3_TM_WB = 0, K3_TM_WS = 128, K3_TM_ACC = 256;
+// One head's decay data for one row tile, read from its table row in shared memory: the
+// reference token's c2 (0 before the chunk) and whether the tile's decay range is too
+// steep for the row/column factorisation.  Every role derives these identically.
+struct TileDecay {
+  const float *c2, *dt;
+  float c2ref, dcoef;
+  bool steep;
+};
+__device__ __forceinline__ TileDecay tile_decay(const float *row, int Q, int ti, int nblk, int valid) {
+  TileDecay t;
+  t.c2 = row + kTabHdr;
+  t.dt = row + kTabHdr + Q;
+  t.dcoef = row[0];
+  t.c2ref = ti > 0 ? t.c2[128 * ti - 1] : 0.f;
+  const int last = min(valid, 128 * nblk) - 1;
+  t.steep = !(fabsf(t.c2ref - t.c2[last]) < kSteepLog2);  // also catches NaN
+  return t;
+}
+
+// TMEM columns: W_base (bf16 pairs, 64 columns per 128-token source block), then two
+// accumulator buffers of [inter 64 | intra, source block 0: 64 | intra, source block 1: 64]
+// columns.  G (fp32, 128 * nblk columns) occupies the buffers until W_base has been built
+// from it.  A steep head builds its own W in the other head's buffer (see below).
+//
+// One thread issues a tcgen05.mma about every 110 ns whatever N is (up to 256), and several
+// issuing threads with their own accumulators run concurrently, so the products of a head
+// are spread over up to three issuers of at most 8 MMAs each: C h_prev^T (warp 1), the
+// intra-chunk product of source block 0 (warp 15) and of source block 1 (warp 16).
+constexpr uint32_t K3_TM_WB = 0, K3_TM_BUF = 128, K3_BUF_COLS = 192;
+__device__ __forceinline__ uint32_t k3_buf(int a) { return K3_TM_BUF + K3_BUF_COLS * (uint32_t)a; }
 
 __global__ void __launch_bounds__(K3_THREADS, 1)
 k_chunk_scan_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_C,
                 const __grid_constant__ CUtensorMap tm_B, const __grid_constant__ CUtensorMap tm_h,
-                const __grid_constant__ CUtensorMap tm_y, const float *__restrict__ dt, const float *__restrict__ A,
-                const float *__restrict__ D, int *err, Dims d, int Q, int nc, int kb0, int nhb0, int kb1, int nhb1) {
+                const __grid_constant__ CUtensorMap tm_y, const float *__restrict__ tab, int *err, Dims d, int Q, int nc,
+                int kb0, int nhb0, int kb1, int nhb1) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   K3Misc *ms = reinterpret_cast<K3Misc *>(base + K3Smem::misc);
@@ -496,14 +536,14 @@ k_chunk_scan_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
     for (int s = 0; s < K3_MAXSLOTS; ++s) {
       mbar_init(&ms->x_full[s], 1);
       mbar_init(&ms->ops_ready[s], 1);
-      mbar_init(&ms->x_free[s], 2);  // commits of both MMA issuers
+      mbar_init(&ms->x_free[s], nblk + 1);  // commits of every MMA issuer
     }
     for (int a = 0; a < 2; ++a) {
-      mbar_init(&ms->acc_full[a], 2);  // commits of both MMA issuers
+      mbar_init(&ms->acc_full[a], nblk + 1);  // commits of every MMA issuer
       mbar_init(&ms->acc_free[a], 1);
     }
     for (int s = 0; s < K3_CUMBUF; ++s) {
-      mbar_init(&ms->cum_full[s], 1);
+      mbar_init(&ms->tab_full[s], 1);
       mbar_init(&ms->cum_free[s], 2);  // x/W warps + output warps
     }
     ms->abort_flag = 0;
@@ -575,9 +615,6 @@ k_chunk_scan_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------- MMA issuer: G, then ACC_inter
-    // A single thread issues one tcgen05.mma about every 65 ns whatever N is up to 128, so
-    // the inter-chunk and intra-chunk products are issued by two warps (this one and warp 15)
-    // into their own accumulators; each commits to acc_full and x_free (count 2).
     if (lane == 0) {
       const uint32_t cm = smem_u32(base + K3Smem::cm), bmm = smem_u32(base + K3Smem::bm(nblk));
       bool ok = mbar_wait(&ms->cb_full, 0, abort_flag, err);
@@ -588,19 +625,24 @@ k_chunk_scan_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
         for (int ks = 0; ks < 8; ++ks) {
           const uint64_t ad = smem_desc_sw128(cm + (ks >> 2) * 16384u + (ks & 3) * 32u, 16u, 1024u);
           const uint64_t bd = smem_desc_sw128(bmm + (ks >> 2) * (uint32_t)nblk * 16384u + (ks & 3) * 32u, 16u, 1024u);
-          mma_bf16(tmem + K3_TM_ACC, ad, bd, idg, ks > 0 ? 1u : 0u);
+          mma_bf16(tmem + K3_TM_BUF, ad, bd, idg, ks > 0 ? 1u : 0u);
         }
         mma_commit(&ms->g_full);
       }
       // G occupies the accumulator columns until W_base has been built from it
       ok = ok && mbar_wait(&ms->w_ready, 0, abort_flag, err);
       const uint32_t id_inter = idesc_bf16_f32(128, TP, false, false);
+      bool prev_steep = false;
       for (int k = 0; ok && k < nh; ++k) {
-        const int s = k % NS, u = k / NS, a = k & 1;
+        const int s = k % NS, u = k / NS, a = k & 1, cb = k % K3_CUMBUF;
         if (!mbar_wait(&ms->x_full[s], u & 1, abort_flag, err)) break;
         if (k >= 2 && !mbar_wait(&ms->acc_free[a], ((k >> 1) - 1) & 1, abort_flag, err)) break;
+        // a steep head k-1 keeps its own W in this head's buffer until its MMAs are done
+        if (prev_steep && !mbar_wait(&ms->x_free[(k - 1) % NS], ((k - 1) / NS) & 1, abort_flag, err)) break;
+        if (!mbar_wait(&ms->tab_full[cb], (k / K3_CUMBUF) & 1, abort_flag, err)) break;
+        prev_steep = tile_decay(ms->tab[cb], Q, ti, nblk, valid).steep;
         tc_fence_after();
-        const uint32_t acc = tmem + K3_TM_ACC + 128u * a;
+        const uint32_t acc = tmem + k3_buf(a);
         const uint32_t so = smem_u32(base + K3Smem::slot(nblk, s));
         const uint32_t hsa = so + (uint32_t)nblk * 16384u;
         // ACC_inter = C_tile h_prev^T: K = d_state
@@ -637,7 +679,7 @@ k_chunk_scan_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
             for (int e = 0; e < 16; ++e) pk[e] = 0u;
           } else {
             float gg[32];
-            tmem_ld32(tmem + lane_off + K3_TM_ACC + (uint32_t)col0, gg);
+            tmem_ld32(tmem + lane_off + K3_TM_BUF + (uint32_t)col0, gg);
             tmem_ld_wait();
             if (jj == ti && grp == q) {
 #pragma unroll
@@ -653,19 +695,22 @@ k_chunk_scan_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
     tc_fence_before();
     named_barrier(1, 128);
     if (tid == 0 && ok) mbar_arrive(&ms->w_ready);
+    bool prev_steep = false;
     for (int k = 0; k < nh; ++k) {
       const int cb = k % K3_CUMBUF, s = k % NS, a = k & 1;
-      const float dh = D[h0 + k];
-      ok = ok && mbar_wait(&ms->cum_full[cb], (k / K3_CUMBUF) & 1, abort_flag, err);
-      const bool steep = ok && ms->steep[cb];
+      ok = ok && mbar_wait(&ms->tab_full[cb], (k / K3_CUMBUF) & 1, abort_flag, err);
+      const TileDecay td = tile_decay(ms->tab[cb], Q, ti, nblk, valid);
+      const float dh = td.dcoef;
+      const bool steep = ok && td.steep;
+      const uint32_t ws_col = k3_buf(a ^ 1);  // a steep head's own W: the other head's buffer
       if (steep) {
-        // the head's own W, from W_base and the full decay; W_steep is free once the MMAs of
-        // head k-1 (the last that may have read it) are complete
-        if (k >= 1) ok = mbar_wait(&ms->x_free[(k - 1) % NS], ((k - 1) / NS) & 1, abort_flag, err);
+        // the head's own W, from W_base and the full decay, built in the buffer of head k-1
+        // once the output warps have read that head's accumulators
+        if (k >= 1) ok = mbar_wait(&ms->acc_free[a ^ 1], ((k - 1) >> 1) & 1, abort_flag, err);
         tc_fence_after();
         if (ok) {
-          const float *c2 = ms->c2[cb];
-          const float *dts = ms->dts[cb];
+          const float *c2 = td.c2;
+          const float *dts = td.dt;
           const float c2t = c2[t];
           for (int jj = 0; jj < nblk; ++jj)
             for (int grp = 0; grp < 4; ++grp) {
@@ -686,9 +731,8 @@ k_chunk_scan_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                 if (jj < ti) {
                   // an earlier block: the reference-token factors (both <= 1 for a decaying head)
                   const float uf = ex2(c2t - c2[r]);
-                  const float *vf = ms->v[cb] + col0;
 #pragma unroll
-                  for (int e = 0; e < 32; ++e) gg[e] *= vf[e] * uf;
+                  for (int e = 0; e < 32; ++e) gg[e] *= ex2(td.c2ref - c2[col0 + e]) * dts[col0 + e] * uf;
                 } else {
                   // the tile's own block: one exp of a difference per element (never overflows)
 #pragma unroll
@@ -700,7 +744,7 @@ k_chunk_scan_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
 #pragma unroll
                 for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(gg[2 * e], gg[2 * e + 1]);
               }
-              tmem_st16(tmem + lane_off + K3_TM_WS + (uint32_t)(64 * jj + 16 * grp), pk);
+              tmem_st16(tmem + lane_off + ws_col + (uint32_t)(64 * jj + 16 * grp), pk);
             }
           tmem_st_wait();
         }
@@ -711,15 +755,20 @@ k_chunk_scan_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
       // head is steep (its W holds the decay), it scales the row by v_s in place.
       ok = ok && mbar_wait(&ms->x_full[s], (k / NS) & 1, abort_flag, err);
       if (k >= 2) ok = ok && mbar_wait(&ms->acc_free[a], ((k >> 1) - 1) & 1, abort_flag, err);
+      // a steep head k-1 keeps its own W in this head's buffer until its MMAs are done
+      if (prev_steep) ok = ok && mbar_wait(&ms->x_free[(k - 1) % NS], ((k - 1) / NS) & 1, abort_flag, err);
+      prev_steep = steep;
       tc_fence_after();
       if (ok) {
         const uint32_t xs = smem_u32(base + K3Smem::slot(nblk, s));
-        const float c2t = ms->c2[cb][t];
-        const float dsc = steep ? dh : dh * ex2(ms->c2ref[cb] - c2t);  // D / u_t
-        const uint32_t acc_i = tmem + lane_off + K3_TM_ACC + 128u * a + 64u;
+        const float c2t = td.c2[t];
+        const float dsc = steep ? dh : dh * ex2(td.c2ref - c2t);  // D / u_t
+        const uint32_t acc_i = tmem + lane_off + k3_buf(a) + 64u;
         for (int jj = 0; jj < nblk; ++jj) {
           const uint32_t ra = xs + (uint32_t)jj * 16384u + (uint32_t)tl * 128u;
-          const float vv = ms->v[cb][128 * jj + tl];
+          // the column factor in bf16: one packed multiply per pair of channels
+          const float vs = ex2(td.c2ref - td.c2[128 * jj + tl]) * td.dt[128 * jj + tl];
+          const uint32_t vv2 = pack_bf16x2(vs, vs);
 #pragma unroll
           for (int half = 0; half < 2; ++half) {  // channels 32 half .. 32 half + 31
             uint32_t w[16];
@@ -748,10 +797,7 @@ k_chunk_scan_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
               for (int cc = 0; cc < 4; ++cc) {
                 uint32_t o4[4];
 #pragma unroll
-                for (int m = 0; m < 4; ++m) {
-                  const uint32_t wv = w[4 * cc + m];
-                  o4[m] = pack_bf16x2(__uint_as_float(wv << 16) * vv, __uint_as_float(wv & 0xffff0000u) * vv);
-                }
+                for (int m = 0; m < 4; ++m) o4[m] = mul_bf16x2(w[4 * cc + m], vv2);
                 st_shared_v4(ra + ((uint32_t)((4 * half + cc) ^ (tl & 7)) << 4), o4[0], o4[1], o4[2], o4[3]);
               }
             }
@@ -782,18 +828,25 @@ k_chunk_scan_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
     const uint32_t srow = smem_u32(stg) + (uint32_t)lane * 128u;
     for (int k = 0; k < nh; ++k) {
       const int a = k & 1, cb = k % K3_CUMBUF, h = h0 + k;
-      bool ok = mbar_wait(&ms->cum_full[cb], (k / K3_CUMBUF) & 1, abort_flag, err);
+      bool ok = mbar_wait(&ms->tab_full[cb], (k / K3_CUMBUF) & 1, abort_flag, err);
       ok = ok && mbar_wait(&ms->acc_full[a], (k >> 1) & 1, abort_flag, err);
       tc_fence_after();
       float vi[32], va[32];
       float et = 0.f, ut = 0.f;
       if (ok) {
-        const uint32_t acc = tmem + lane_off + K3_TM_ACC + 128u * a + 32u * hf;
-        tmem_ld32(acc, vi);
+        const uint32_t acc = tmem + lane_off + k3_buf(a) + 32u * hf;
         tmem_ld32(acc + 64u, va);
-        const float c2t = ms->c2[cb][t];
+        if (nblk > 1) {  // the two source blocks' intra-chunk products share the row factor u_t
+          tmem_ld32(acc + 128u, vi);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 32; ++j) va[j] += vi[j];
+        }
+        tmem_ld32(acc, vi);
+        const TileDecay td = tile_decay(ms->tab[cb], Q, ti, nblk, valid);
+        const float c2t = td.c2[t];
         et = ex2(c2t);
-        ut = ms->steep[cb] ? 1.f : ex2(c2t - ms->c2ref[cb]);
+        ut = td.steep ? 1.f : ex2(c2t - td.c2ref);
         tmem_ld_wait();
       }
       // the accumulators and decay tables are read: release them before writing y
@@ -824,89 +877,56 @@ k_chunk_scan_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
     }
     if (lane == 0) tma_store_wait_all();
     __syncwarp();
-  } else if (warp == 15) {
-    // ------------------------------------------------------------- MMA issuer: ACC_intra
-    // ops_ready implies x_full, acc_free and W_base: the scaling warps waited for all three
-    // before storing D x / u into the accumulator this MMA adds onto.
-    if (lane == 0) {
+  } else if (warp == 15 || warp == 16) {
+    // ------------------------------------------------------------- MMA issuers: ACC_intra
+    // Warp 15 forms W_{., 0} X'_0 onto D x / u (stored by the scaling warps), warp 16 the
+    // second row tile's W_{., 1} X'_1 into its own accumulator.  ops_ready implies x_full,
+    // acc_free and W_base: the scaling warps waited for all three.
+    const int jj = warp - 15;  // source block
+    if (lane == 0 && jj < nblk) {
       const uint32_t id_intra = idesc_bf16_f32(128, TP, false, true);
       for (int k = 0; k < nh; ++k) {
         const int s = k % NS, u = k / NS, a = k & 1, cb = k % K3_CUMBUF;
         if (!mbar_wait(&ms->ops_ready[s], u & 1, abort_flag, err)) break;
+        if (!mbar_wait(&ms->tab_full[cb], (k / K3_CUMBUF) & 1, abort_flag, err)) break;  // complete already
         tc_fence_after();
-        const uint32_t acc = tmem + K3_TM_ACC + 128u * a;
+        const uint32_t acc = tmem + k3_buf(a) + 64u * (uint32_t)(1 + jj);
         const uint32_t so = smem_u32(base + K3Smem::slot(nblk, s));
-        // ACC_intra += W X': A from TMEM (W_base, or the head's own W when steep), K = source tokens
-        const uint32_t wa = tmem + (ms->steep[cb] ? K3_TM_WS : K3_TM_WB);
-        for (int jj = 0; jj < nblk; ++jj)
-          for (int ks = 0; ks < 8; ++ks) {
-            const uint64_t bd = smem_desc_sw128(so + jj * 16384u + ks * 2048u, 16384u, 1024u);
-            mma_bf16_ts(acc + 64, wa + (uint32_t)(64 * jj + 8 * ks), bd, id_intra, 1u);  // onto D x / u
-          }
+        // A from TMEM (W_base, or a steep head's own W in the other buffer), K = source tokens
+        const bool steep = tile_decay(ms->tab[cb], Q, ti, nblk, valid).steep;
+        const uint32_t wa = tmem + (steep ? k3_buf(a ^ 1) : K3_TM_WB) + (uint32_t)(64 * jj);
+        for (int ks = 0; ks < 8; ++ks) {
+          const uint64_t bd = smem_desc_sw128(so + jj * 16384u + ks * 2048u, 16384u, 1024u);
+          // block 0 adds onto D x / u; block 1 starts its own accumulator
+          mma_bf16_ts(acc, wa + (uint32_t)(8 * ks), bd, id_intra, (jj == 0 || ks > 0) ? 1u : 0u);
+        }
         mma_commit(&ms->acc_full[a]);
         mma_commit(&ms->x_free[s]);
       }
     }
     __syncwarp();
-  } else {
-    // ------------------------------------------------------------- decay-table warp
-    // dt and A of head k + 1 are loaded while head k's buffer is awaited and filled
-    const int per = Q / 32;
-    auto load_head = [&](int k, float (&v)[8], float &a) {
-      const int h = h0 + k;
-      a = A[h];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int tt = lane * per + j;
-        v[j] = (j < per && tt < valid) ? dt[((size_t)bi * d.L + t0 + tt) * d.H + h] : 0.f;
+  } else if (warp == 14) {
+    // ------------------------------------------------------------- decay-table loads
+    // One bulk copy per head of its table row (written by the cumulative-sum kernel) into a
+    // ring of K3_CUMBUF entries, released by the scaling and the output warps.
+    if (lane == 0) {
+      const uint32_t tab_bytes = (uint32_t)tab_row_floats(Q) * 4u;
+      const float *row0 = tab + (((size_t)bi * d.H + h0) * nc + c) * (size_t)tab_row_floats(Q);
+      const size_t head_stride = (size_t)nc * tab_row_floats(Q);
+      grid_dep_wait();
+      int issued = 0;
+      for (int k = 0; k < nh; ++k) {
+        const int cb = k % K3_CUMBUF;
+        if (k >= K3_CUMBUF && !mbar_wait(&ms->cum_free[cb], ((k / K3_CUMBUF) - 1) & 1, abort_flag, err)) break;
+        mbar_arrive_expect_tx(&ms->tab_full[cb], tab_bytes);
+        bulk_load(ms->tab[cb], row0 + k * head_stride, tab_bytes, &ms->tab_full[cb]);
+        issued = k + 1;
       }
-    };
-    float dtv[8], dtn[8], acur = 0.f, anxt = 0.f;
-    if (nh > 0) load_head(0, dtv, acur);
-    for (int k = 0; k < nh; ++k) {
-      const int cb = k % K3_CUMBUF;
-      if (k + 1 < nh) load_head(k + 1, dtn, anxt);
-      if (k >= K3_CUMBUF && !mbar_wait(&ms->cum_free[cb], ((k / K3_CUMBUF) - 1) & 1, abort_flag, err)) break;
-      const float a2 = acur * kLog2e;
-      float c2v[8];
-      float run = 0.f;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        run += dtv[j] * a2;
-        c2v[j] = run;
-      }
-      float incl = run;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const float vv = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += vv;
-      }
-      const float excl = incl - run;
-      float *c2 = ms->c2[cb];
-      float *dts = ms->dts[cb];
-#pragma unroll
-      for (int j = 0; j < 8; ++j)
-        if (j < per) {
-          c2[lane * per + j] = c2v[j] + excl;
-          dts[lane * per + j] = dtv[j];
-        }
-      __syncwarp();
-      const int ncol = 128 * nblk;
-      const int last = min(valid, ncol) - 1;
-      const float c2r = (ti > 0) ? c2[128 * ti - 1] : 0.f;
-      const float range = fabsf(c2r - c2[last]);
-      const int steep = !(range < kSteepLog2);  // also catches NaN
-      for (int sidx = lane; sidx < ncol; sidx += 32) ms->v[cb][sidx] = ex2(c2r - c2[sidx]) * dts[sidx];
-      if (lane == 0) {
-        ms->steep[cb] = steep;
-        ms->c2ref[cb] = c2r;
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&ms->cum_full[cb]);
-#pragma unroll
-      for (int j = 0; j < 8; ++j) dtv[j] = dtn[j];
-      acur = anxt;
+      if (*abort_flag)  // let this CTA's own copies land before it exits
+        for (int k = (issued > K3_CUMBUF ? issued - K3_CUMBUF : 0); k < issued; ++k)
+          mbar_wait_drain(&ms->tab_full[k % K3_CUMBUF], (k / K3_CUMBUF) & 1);
     }
+    __syncwarp();
   }
 
   tc_fence_before();
@@ -982,18 +1002,19 @@ int pick_heads_per_cta(int base_items, int hpg, int sms, double overhead) {
   return best_kb;
 }
 
-// Head split of the chunk-scan kernel.  A CTA of the second row tile costs about 1.5x a
-// first-tile CTA per head (twice the x tile and the in-chunk product); each also pays a
-// fixed set-up (about 1.8 heads).  Candidate splits are scored by simulating the
-// hardware's greedy, in-order placement of CTAs onto SMs (one CTA per SM at a time).
+// Head split of the chunk-scan kernel.  A CTA of the second row tile costs about 1.26x a
+// first-tile CTA per head (twice the x tile and the in-chunk product; measured); each also
+// pays a fixed set-up of about 1.8 first-tile heads.  Every pair of head-block sizes is
+// scored by simulating the hardware's greedy, in-order placement of CTAs onto SMs (one
+// CTA per SM at a time); ties go to the split with fewer CTAs.
 struct ScanSplit {
   int kb0, nhb0, kb1, nhb1;
 };
 
 double simulate_makespan(int groups, int hpg, int kb0, int kb1, int ntt, int sms) {
-  constexpr double kSetup = 1.8, kTile1 = 1.5;
-  std::vector<double> free_at(sms, 0.0);
-  std::priority_queue<double, std::vector<double>, std::greater<double>> q(free_at.begin(), free_at.end());
+  constexpr double kSetup = 1.8, kTile1 = 1.26;
+  std::priority_queue<double, std::vector<double>, std::greater<double>> q;
+  for (int i = 0; i < sms; ++i) q.push(0.0);
   const int nhb0 = (hpg + kb0 - 1) / kb0, nhb1 = ntt > 1 ? (hpg + kb1 - 1) / kb1 : 0;
   double end = 0.0;
   for (int gi = 0; gi < groups; ++gi)
@@ -1019,14 +1040,24 @@ ScanSplit pick_scan_split(int groups, int hpg, int ntt, int sms) {
   if (it != cache.end()) return it->second;
   ScanSplit best{hpg, 1, hpg, ntt > 1 ? 1 : 0};
   double best_t = 1e300;
-  for (int kb1 = 1; kb1 <= hpg; ++kb1) {
-    const int kb0 = ntt > 1 ? std::min(hpg, std::max(1, (int)std::lround(kb1 * 1.5))) : kb1;
-    const double t = simulate_makespan(groups, hpg, kb0, kb1, ntt, sms);
-    if (t < best_t - 1e-9) {
-      best_t = t;
-      best = {kb0, (hpg + kb0 - 1) / kb0, kb1, ntt > 1 ? (hpg + kb1 - 1) / kb1 : 0};
-    }
+  long best_ctas = 0;
+  // Only block sizes that give a distinct block count are worth scoring.
+  std::vector<int> sizes;
+  for (int nb = 1; nb <= hpg; ++nb) {
+    const int kb = (hpg + nb - 1) / nb;
+    if (sizes.empty() || sizes.back() != kb) sizes.push_back(kb);
   }
+  for (int kb1 : (ntt > 1 ? sizes : std::vector<int>{hpg}))
+    for (int kb0 : sizes) {
+      const int nhb0 = (hpg + kb0 - 1) / kb0, nhb1 = ntt > 1 ? (hpg + kb1 - 1) / kb1 : 0;
+      const long ctas = (long)groups * (nhb0 + nhb1);
+      const double t = simulate_makespan(groups, hpg, kb0, kb1, ntt, sms);
+      if (t < best_t - 1e-9 || (t < best_t + 1e-9 && ctas < best_ctas)) {
+        best_t = t;
+        best_ctas = ctas;
+        best = {kb0, nhb0, kb1, nhb1};
+      }
+    }
   cache[key] = best;
   return best;
 }
@@ -1054,12 +1085,13 @@ cudaError_t launch_after(dim3 grid, unsigned threads, size_t smem, cudaStream_t 
 bool tc_prefill_supported(const Dims &d, int Q) { return d.P == TP && d.N == TN && (Q == 128 || Q == 256); }
 
 size_t tc_prefill_smem_k1(int Q) { return 1024 + K1Smem::misc(Q) + sizeof(K1Misc); }
+size_t tc_prefill_table_floats(const Dims &d, int Q, int nc) { return (size_t)d.b * d.H * nc * tab_row_floats(Q); }
 size_t tc_prefill_smem_k3() { return kK3SmemBytes; }
 
 cudaError_t launch_tc_prefill(const __nv_bfloat16 *x, const float *dt, const float *A, const __nv_bfloat16 *B,
-                              const __nv_bfloat16 *C, const float *D, float *y, float *final_state, float *states,
-                              float *cdecay, __nv_bfloat16 *hprev, int *err, const Dims &d, int Q, int nc,
-                              cudaStream_t st, const cudaEvent_t *ev) {
+                              const __nv_bfloat16 *C, const float *D, float *y, float *final_state, float *tab,
+                              float *states, float *cdecay, __nv_bfloat16 *hprev, int *err, const Dims &d, int Q,
+                              int nc, cudaStream_t st, const cudaEvent_t *ev) {
   CUtensorMap tm_x1, tm_B1, tm_x3, tm_C3, tm_B3, tm_h3, tm_y3;
   const uint64_t HP = (uint64_t)d.H * d.P, GN = (uint64_t)d.G * d.N;
   if (!make_map(&tm_x1, x, HP, d.L, d.b, Q) || !make_map(&tm_B1, B, GN, d.L, d.b, Q) ||
@@ -1070,21 +1102,21 @@ cudaError_t launch_tc_prefill(const __nv_bfloat16 *x, const float *dt, const flo
     return cudaErrorInvalidValue;
   const int sms = num_sms();
   auto mark = [&](int i) { return ev ? cudaEventRecord(ev[i], st) : cudaSuccess; };
-  // Without per-kernel events the three kernels overlap their set-up with the tail of the
-  // one before (programmatic dependent launch); with events between them they run serially.
+  // Without per-kernel events each kernel overlaps its set-up with the tail of the one
+  // before (programmatic dependent launch); with events between them they run serially.
   const bool pdl = ev == nullptr;
   cudaError_t e = mark(0);
   if (e != cudaSuccess) return e;
   // K1
   {
     const int base_items = d.b * nc * d.G;
-    const int kb = pick_heads_per_cta(base_items, d.hpg, sms, 1.0);
+    const int kb = std::min(K1_KB_MAX, pick_heads_per_cta(base_items, d.hpg, sms, 1.0));
     const int nhb = (d.hpg + kb - 1) / kb;
     const size_t smem = tc_prefill_smem_k1(Q);
     e = cudaFuncSetAttribute(k_chunk_state_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    k_chunk_state_tc<<<(unsigned)(base_items * nhb), K1_THREADS, smem, st>>>(tm_x1, tm_B1, dt, A, states, cdecay,
-                                                                             err, d, Q, nc, kb, nhb);
+    k_chunk_state_tc<<<(unsigned)(base_items * nhb), K1_THREADS, smem, st>>>(tm_x1, tm_B1, dt, A, D, tab, cdecay,
+                                                                             states, err, d, Q, nc, kb, nhb);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   if ((e = mark(1)) != cudaSuccess) return e;
@@ -1104,8 +1136,8 @@ cudaError_t launch_tc_prefill(const __nv_bfloat16 *x, const float *dt, const flo
     e = cudaFuncSetAttribute(k_chunk_scan_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kK3SmemBytes);
     if (e != cudaSuccess) return e;
     e = launch_after(dim3((unsigned)(groups * (sp.nhb0 + sp.nhb1))), K3_THREADS, kK3SmemBytes, st, pdl,
-                     k_chunk_scan_tc, tm_x3, tm_C3, tm_B3, tm_h3, tm_y3, dt, A, D, err, d, Q, nc, sp.kb0, sp.nhb0,
-                     sp.kb1, sp.nhb1);
+                     k_chunk_scan_tc, tm_x3, tm_C3, tm_B3, tm_h3, tm_y3, (const float *)tab, err, d, Q, nc, sp.kb0,
+                     sp.nhb0, sp.kb1, sp.nhb1);
     if (e != cudaSuccess) return e;
   }
   return mark(3);

@@ -66,6 +66,7 @@ struct PrefillPlan {
   int nc = 0;             // chunks per sequence
   size_t cum_off = 0;     // SIMT: float [b][H][nc][Q] in-chunk cumulative decay
   size_t states_off = 0;  // both: float [b][nc][H][P][N] chunk states (SIMT: replaced by h_prev)
+  size_t tab_off = 0;     // tensor cores: float [b][H][nc][4 + 2Q] decay table (D, chunk decay, c2, dt)
   size_t cdecay_off = 0;  // tensor cores: float [b][H][nc] total decay of each chunk
   size_t hprev_off = 0;   // tensor cores: bf16 [b][nc][H][P][N] state entering each chunk
   size_t bytes = 0;
@@ -82,7 +83,8 @@ PrefillPlan plan_prefill(const Dims &d, ssd_dtype dtype, int Q) {
     pl.states_off = kAlign;
     pl.cdecay_off = pl.states_off + align_up(nstate * sizeof(float));
     pl.hprev_off = pl.cdecay_off + align_up((size_t)d.b * d.H * pl.nc * sizeof(float));
-    pl.bytes = pl.hprev_off + align_up(nstate * sizeof(__nv_bfloat16));
+    pl.tab_off = pl.hprev_off + align_up(nstate * sizeof(__nv_bfloat16));
+    pl.bytes = pl.tab_off + align_up(ssd::tc_prefill_table_floats(d, Q, pl.nc) * sizeof(float));
     pl.launches = 3;
   } else {
     pl.path = Path::kSimt;
@@ -192,7 +194,8 @@ static ssd_status prefill_impl(const ssd_dims *dims, ssd_dtype dtype, const void
   if (pl.path == Path::kTensorCore)
     return cuda_status(ssd::launch_tc_prefill(
         static_cast<const __nv_bfloat16 *>(x), dt, A, static_cast<const __nv_bfloat16 *>(B),
-        static_cast<const __nv_bfloat16 *>(C), D, y, final_state, reinterpret_cast<float *>(ws + pl.states_off),
+        static_cast<const __nv_bfloat16 *>(C), D, y, final_state, reinterpret_cast<float *>(ws + pl.tab_off),
+        reinterpret_cast<float *>(ws + pl.states_off),
         reinterpret_cast<float *>(ws + pl.cdecay_off), reinterpret_cast<__nv_bfloat16 *>(ws + pl.hprev_off),
         reinterpret_cast<int *>(ws), d, chunk, pl.nc, st, ev));
   if (dtype == SSD_F32)
