@@ -131,6 +131,31 @@ SSD_API ssd_status ssd_prefill(const ssd_dims *dims, ssd_dtype dtype, const void
                        size_t workspace_bytes, ssd_stream_t stream);
 
 /*
+ * ssd_prefill from a given initial state, optionally exporting the state at every chunk
+ * boundary: the carried state of the chunked form ("Engineering Hybrid State-Space
+ * Models" section 2), started from h_{-1} = initial_state instead of zero.  This lets a
+ * long prompt be processed in pieces (pass one piece's final_state as the next piece's
+ * initial_state) and a prefix cache keep the state at any chunk boundary.
+ *
+ *   initial_state  [batch, nheads, headdim, dstate] fp32, or NULL for a zero state.  It
+ *                  may be the same array as final_state (then updated in place); it
+ *                  must not overlap any other argument.
+ *   chunk_states   [batch, nchunks, nheads, headdim, dstate] fp32 with
+ *                  nchunks = ceil(seqlen / chunk), or NULL.  chunk_states[b][c] is the
+ *                  state after token min((c + 1) * chunk, seqlen) - 1, so its last entry
+ *                  equals final_state.  Written only when non-NULL.
+ *
+ * With both NULL this is exactly ssd_prefill.  When seqlen == 0, final_state is set to
+ * initial_state (or zeros) and chunk_states is not touched.  Workspace, alignment (16
+ * bytes for both optional arrays), asynchrony and errors as ssd_prefill;
+ * SSD_ERR_INVALID_ARG also for a misaligned initial_state or chunk_states.
+ */
+SSD_API ssd_status ssd_prefill_ex(const ssd_dims *dims, ssd_dtype dtype, const void *x, const float *dt,
+                                  const float *A, const void *B, const void *C, const float *D, int chunk,
+                                  const float *initial_state, float *y, float *final_state, float *chunk_states,
+                                  void *workspace, size_t workspace_bytes, ssd_stream_t stream);
+
+/*
  * ssd_prefill, with per-kernel timing for profiling harnesses.  `events` holds
  * num_events caller-created cudaEvent_t handles (cudaEventDefault flags, i.e. timing
  * enabled), num_events >= ssd_prefill_kernel_launches() + 1.  events[i] is recorded on

@@ -15,8 +15,9 @@ cudaError_t launch_dA_cumsum(const float *dt, const float *A, float *cum, const 
 template <typename T>
 cudaError_t launch_chunk_state_simt(const T *x, const float *dt, const T *B, const float *cum, float *states,
                                     const Dims &d, int Q, int nc, cudaStream_t st);
-cudaError_t launch_state_passing(float *states, const float *cum, float *final_state, const Dims &d, int Q,
-                                 int nc, cudaStream_t st);
+// init: state before the first token (NULL: zero); cstates: state after each chunk (NULL: not written)
+cudaError_t launch_state_passing(float *states, const float *cum, const float *init, float *final_state,
+                                 float *cstates, const Dims &d, int Q, int nc, cudaStream_t st);
 template <typename T>
 cudaError_t launch_chunk_scan_simt(const T *x, const float *dt, const T *B, const T *C, const float *D,
                                    const float *cum, const float *hprev, float *y, const Dims &d, int Q, int nc,
@@ -28,9 +29,9 @@ bool tc_prefill_supported(const Dims &d, int Q);
 // floats of the per-(batch, head, chunk) decay table the tensor-core kernels share
 size_t tc_prefill_table_floats(const Dims &d, int Q, int nc);
 cudaError_t launch_tc_prefill(const __nv_bfloat16 *x, const float *dt, const float *A, const __nv_bfloat16 *B,
-                              const __nv_bfloat16 *C, const float *D, float *y, float *final_state, float *tab,
-                              float *states, float *cdecay, __nv_bfloat16 *hprev, int *err, const Dims &d, int Q,
-                              int nc, cudaStream_t st, const cudaEvent_t *ev);
+                              const __nv_bfloat16 *C, const float *D, const float *init, float *y, float *final_state,
+                              float *cstates, float *tab, float *states, float *cdecay, __nv_bfloat16 *hprev, int *err,
+                              const Dims &d, int Q, int nc, cudaStream_t st, const cudaEvent_t *ev);
 
 // decode.cu
 template <typename T>

@@ -110,10 +110,12 @@ k_chunk_state_simt(const T *__restrict__ x, const float *__restrict__ dt, const 
 
 // ------------------------------------------------------------------------ (c)
 // grid (b * H, ceil(P*N/4 / 256)), block 256: one float4 of the state per thread,
-// sequential over chunks.
+// sequential over chunks.  The recurrence starts from `init` (zero if NULL); with
+// `cstates` non-NULL the state after every chunk is also written there.  `init` may be
+// final_state: each thread reads its element before it writes it.
 __global__ void __launch_bounds__(256)
-k_state_passing(float *__restrict__ states, const float *__restrict__ cum,
-                float *__restrict__ final_state, Dims d, int Q, int nc) {
+k_state_passing(float *__restrict__ states, const float *__restrict__ cum, const float *init,
+                float *final_state, float *__restrict__ cstates, Dims d, int Q, int nc) {
   const int PN4 = d.P * d.N / 4;
   const int e = blockIdx.y * blockDim.x + threadIdx.x;
   const int h = blockIdx.x % d.H, bi = blockIdx.x / d.H;
@@ -121,7 +123,9 @@ k_state_passing(float *__restrict__ states, const float *__restrict__ cum,
   const float *cumh = cum + ((size_t)bi * d.H + h) * nc * Q;
   const size_t chunk_stride4 = (size_t)d.H * PN4;  // float4s between consecutive chunks
   float4 *sp = reinterpret_cast<float4 *>(states) + ((size_t)bi * nc * d.H + h) * PN4 + e;
-  float4 hs = make_float4(0.f, 0.f, 0.f, 0.f);
+  const size_t own4 = ((size_t)bi * d.H + h) * PN4 + e;  // this element in a [b][H][P][N] state
+  float4 hs = init ? reinterpret_cast<const float4 *>(init)[own4] : make_float4(0.f, 0.f, 0.f, 0.f);
+  float4 *cs = cstates ? reinterpret_cast<float4 *>(cstates) + ((size_t)bi * nc * d.H + h) * PN4 + e : nullptr;
   float4 s = sp[0];
   for (int c = 0; c < nc; ++c) {
     const float4 s_next = (c + 1 < nc) ? sp[(c + 1) * chunk_stride4] : make_float4(0.f, 0.f, 0.f, 0.f);
@@ -131,9 +135,10 @@ k_state_passing(float *__restrict__ states, const float *__restrict__ cum,
     hs.y = fmaf(dec, hs.y, s.y);
     hs.z = fmaf(dec, hs.z, s.z);
     hs.w = fmaf(dec, hs.w, s.w);
+    if (cs) cs[c * chunk_stride4] = hs;  // state after chunk c
     s = s_next;
   }
-  reinterpret_cast<float4 *>(final_state)[((size_t)bi * d.H + h) * PN4 + e] = hs;
+  reinterpret_cast<float4 *>(final_state)[own4] = hs;
 }
 
 // ------------------------------------------------------------------------ (d)
@@ -288,10 +293,11 @@ cudaError_t launch_chunk_state_simt(const T *x, const float *dt, const T *B, con
   return cudaGetLastError();
 }
 
-cudaError_t launch_state_passing(float *states, const float *cum, float *final_state, const Dims &d,
-                                 int Q, int nc, cudaStream_t st) {
+cudaError_t launch_state_passing(float *states, const float *cum, const float *init, float *final_state,
+                                 float *cstates, const Dims &d, int Q, int nc, cudaStream_t st) {
   const int PN4 = d.P * d.N / 4;
-  k_state_passing<<<dim3(d.b * d.H, (PN4 + 255) / 256), 256, 0, st>>>(states, cum, final_state, d, Q, nc);
+  k_state_passing<<<dim3(d.b * d.H, (PN4 + 255) / 256), 256, 0, st>>>(states, cum, init, final_state, cstates, d, Q,
+                                                                        nc);
   return cudaGetLastError();
 }
 

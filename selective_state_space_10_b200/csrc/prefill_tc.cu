@@ -361,11 +361,15 @@ k_chunk_state_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
 // grid (b * H, ceil(P*N/4 / 256)), block 256: one float4 of the state per thread.  The
 // chunk states of 8 chunks are loaded before the sequential update so that their
 // latencies overlap; the state entering chunk c is stored in bf16, the final state in fp32.
+// The recurrence starts from `init` (zero if NULL); with `cstates` non-NULL the state
+// after every chunk is also written there in fp32.  `init` may be final_state: each
+// thread reads its element before it writes it.
 constexpr int K2_BATCH = 8;
 
 __global__ void __launch_bounds__(256)
 k_state_passing_bf16(const float *__restrict__ states, const float *__restrict__ cdecay,
-                     __nv_bfloat16 *__restrict__ hprev, float *__restrict__ final_state, Dims d, int nc) {
+                     __nv_bfloat16 *__restrict__ hprev, const float *init, float *final_state,
+                     float *__restrict__ cstates, Dims d, int nc) {
   const int PN4 = d.P * d.N / 4;
   const int e4 = blockIdx.y * blockDim.x + threadIdx.x;
   sm100::grid_dep_launch();  // the chunk scan may start its own set-up meanwhile
@@ -377,7 +381,9 @@ k_state_passing_bf16(const float *__restrict__ states, const float *__restrict__
   const float4 *sp = reinterpret_cast<const float4 *>(states) + off0;
   uint2 *hp = reinterpret_cast<uint2 *>(hprev) + off0;
   const float *dec = cdecay + ((size_t)bi * d.H + h) * nc;
-  float4 hs = make_float4(0.f, 0.f, 0.f, 0.f);
+  const size_t own4 = ((size_t)bi * d.H + h) * PN4 + e4;  // this element in a [b][H][P][N] state
+  float4 hs = init ? reinterpret_cast<const float4 *>(init)[own4] : make_float4(0.f, 0.f, 0.f, 0.f);
+  float4 *cs = cstates ? reinterpret_cast<float4 *>(cstates) + off0 : nullptr;
   for (int c0 = 0; c0 < nc; c0 += K2_BATCH) {
     float4 sv[K2_BATCH];
     float dc[K2_BATCH];
@@ -395,9 +401,10 @@ k_state_passing_bf16(const float *__restrict__ states, const float *__restrict__
         hs.y = fmaf(dc[j], hs.y, sv[j].y);
         hs.z = fmaf(dc[j], hs.z, sv[j].z);
         hs.w = fmaf(dc[j], hs.w, sv[j].w);
+        if (cs) cs[(size_t)(c0 + j) * cstride] = hs;  // state after chunk c0 + j
       }
   }
-  reinterpret_cast<float4 *>(final_state)[((size_t)bi * d.H + h) * PN4 + e4] = hs;
+  reinterpret_cast<float4 *>(final_state)[own4] = hs;
 }
 
 // ============================================================================ K3
@@ -1089,9 +1096,9 @@ size_t tc_prefill_table_floats(const Dims &d, int Q, int nc) { return (size_t)d.
 size_t tc_prefill_smem_k3() { return kK3SmemBytes; }
 
 cudaError_t launch_tc_prefill(const __nv_bfloat16 *x, const float *dt, const float *A, const __nv_bfloat16 *B,
-                              const __nv_bfloat16 *C, const float *D, float *y, float *final_state, float *tab,
-                              float *states, float *cdecay, __nv_bfloat16 *hprev, int *err, const Dims &d, int Q,
-                              int nc, cudaStream_t st, const cudaEvent_t *ev) {
+                              const __nv_bfloat16 *C, const float *D, const float *init, float *y, float *final_state,
+                              float *cstates, float *tab, float *states, float *cdecay, __nv_bfloat16 *hprev, int *err,
+                              const Dims &d, int Q, int nc, cudaStream_t st, const cudaEvent_t *ev) {
   CUtensorMap tm_x1, tm_B1, tm_x3, tm_C3, tm_B3, tm_h3, tm_y3;
   const uint64_t HP = (uint64_t)d.H * d.P, GN = (uint64_t)d.G * d.N;
   if (!make_map(&tm_x1, x, HP, d.L, d.b, Q) || !make_map(&tm_B1, B, GN, d.L, d.b, Q) ||
@@ -1124,7 +1131,7 @@ cudaError_t launch_tc_prefill(const __nv_bfloat16 *x, const float *dt, const flo
   {
     const int per_head = d.P * d.N / 4;
     e = launch_after(dim3(d.b * d.H, (per_head + 255) / 256), 256, 0, st, pdl, k_state_passing_bf16, states, cdecay,
-                     hprev, final_state, d, nc);
+                     hprev, init, final_state, cstates, d, nc);
     if (e != cudaSuccess) return e;
   }
   if ((e = mark(2)) != cudaSuccess) return e;

@@ -108,8 +108,8 @@ struct Marker {
 
 template <typename T>
 ssd_status run_prefill(const Dims &d, int Q, const PrefillPlan &pl, const T *x, const float *dt,
-                       const float *A, const T *B, const T *C, const float *D, float *y, float *final_state,
-                       char *ws, cudaStream_t st, cudaEvent_t const *ev) {
+                       const float *A, const T *B, const T *C, const float *D, const float *init, float *y,
+                       float *final_state, float *cstates, char *ws, cudaStream_t st, cudaEvent_t const *ev) {
   float *cum = reinterpret_cast<float *>(ws + pl.cum_off);
   float *states = reinterpret_cast<float *>(ws + pl.states_off);
   Marker m{ev, st};
@@ -118,7 +118,7 @@ ssd_status run_prefill(const Dims &d, int Q, const PrefillPlan &pl, const T *x, 
   if (e == cudaSuccess) e = m.mark();
   if (e == cudaSuccess) e = ssd::launch_chunk_state_simt<T>(x, dt, B, cum, states, d, Q, pl.nc, st);
   if (e == cudaSuccess) e = m.mark();
-  if (e == cudaSuccess) e = ssd::launch_state_passing(states, cum, final_state, d, Q, pl.nc, st);
+  if (e == cudaSuccess) e = ssd::launch_state_passing(states, cum, init, final_state, cstates, d, Q, pl.nc, st);
   if (e == cudaSuccess) e = m.mark();
   if (e == cudaSuccess) e = ssd::launch_chunk_scan_simt<T>(x, dt, B, C, D, cum, states, y, d, Q, pl.nc, st);
   if (e == cudaSuccess) e = m.mark();
@@ -161,9 +161,10 @@ int ssd_prefill_kernel_launches(const ssd_dims *dims, ssd_dtype dtype, int chunk
 }
 
 static ssd_status prefill_impl(const ssd_dims *dims, ssd_dtype dtype, const void *x, const float *dt,
-                               const float *A, const void *B, const void *C, const float *D, int chunk, float *y,
-                               float *final_state, void *workspace, size_t workspace_bytes, ssd_stream_t stream,
-                               void *const *events, int num_events, bool timed) {
+                               const float *A, const void *B, const void *C, const float *D, int chunk,
+                               const float *init, float *y, float *final_state, float *cstates, void *workspace,
+                               size_t workspace_bytes, ssd_stream_t stream, void *const *events, int num_events,
+                               bool timed) {
   Dims d;
   ssd_status s = check_dims(dims, dtype, true, &d);
   if (s != SSD_OK) return s;
@@ -172,6 +173,10 @@ static ssd_status prefill_impl(const ssd_dims *dims, ssd_dtype dtype, const void
   const int64_t nx = ntok * d.H * d.P, nbc = ntok * d.G * d.N, nst = (int64_t)d.b * d.H * d.P * d.N;
   if (!check_ptr(x, nx, 16) || !check_ptr(B, nbc, 16) || !check_ptr(C, nbc, 16) || !check_ptr(y, nx, 16) ||
       !check_ptr(dt, ntok * d.H, 4) || !check_ptr(final_state, nst, 16))
+    return SSD_ERR_INVALID_ARG;
+  // optional arrays: NULL means "none"; when given they must be aligned
+  const int64_t ncs = (int64_t)d.b * ((d.L + chunk - 1) / chunk) * d.H * d.P * d.N;
+  if ((init != nullptr && !check_ptr(init, nst, 16)) || (cstates != nullptr && !check_ptr(cstates, ncs, 16)))
     return SSD_ERR_INVALID_ARG;
   const bool any_heads = d.b > 0 && d.L > 0;
   if (!check_ptr(A, any_heads ? d.H : 0, 4) || !check_ptr(D, any_heads ? d.H : 0, 4)) return SSD_ERR_INVALID_ARG;
@@ -186,7 +191,11 @@ static ssd_status prefill_impl(const ssd_dims *dims, ssd_dtype dtype, const void
 
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (d.b == 0) return SSD_OK;
-  if (d.L == 0) return cuda_status(cudaMemsetAsync(final_state, 0, (size_t)nst * sizeof(float), st));
+  if (d.L == 0) {  // no tokens: the final state is the initial one
+    if (init == nullptr) return cuda_status(cudaMemsetAsync(final_state, 0, (size_t)nst * sizeof(float), st));
+    if (init == final_state) return SSD_OK;
+    return cuda_status(cudaMemcpyAsync(final_state, init, (size_t)nst * sizeof(float), cudaMemcpyDeviceToDevice, st));
+  }
   char *ws = static_cast<char *>(workspace);
   cudaEvent_t const *ev = timed ? reinterpret_cast<cudaEvent_t const *>(events) : nullptr;
   cudaError_t e = cudaMemsetAsync(ws, 0, sizeof(int), st);  // device error word
@@ -194,31 +203,39 @@ static ssd_status prefill_impl(const ssd_dims *dims, ssd_dtype dtype, const void
   if (pl.path == Path::kTensorCore)
     return cuda_status(ssd::launch_tc_prefill(
         static_cast<const __nv_bfloat16 *>(x), dt, A, static_cast<const __nv_bfloat16 *>(B),
-        static_cast<const __nv_bfloat16 *>(C), D, y, final_state, reinterpret_cast<float *>(ws + pl.tab_off),
+        static_cast<const __nv_bfloat16 *>(C), D, init, y, final_state, cstates, reinterpret_cast<float *>(ws + pl.tab_off),
         reinterpret_cast<float *>(ws + pl.states_off),
         reinterpret_cast<float *>(ws + pl.cdecay_off), reinterpret_cast<__nv_bfloat16 *>(ws + pl.hprev_off),
         reinterpret_cast<int *>(ws), d, chunk, pl.nc, st, ev));
   if (dtype == SSD_F32)
     return run_prefill<float>(d, chunk, pl, static_cast<const float *>(x), dt, A, static_cast<const float *>(B),
-                              static_cast<const float *>(C), D, y, final_state, ws, st, ev);
+                              static_cast<const float *>(C), D, init, y, final_state, cstates, ws, st, ev);
   return run_prefill<__nv_bfloat16>(d, chunk, pl, static_cast<const __nv_bfloat16 *>(x), dt, A,
                                     static_cast<const __nv_bfloat16 *>(B), static_cast<const __nv_bfloat16 *>(C), D,
-                                    y, final_state, ws, st, ev);
+                                    init, y, final_state, cstates, ws, st, ev);
 }
 
 ssd_status ssd_prefill(const ssd_dims *dims, ssd_dtype dtype, const void *x, const float *dt, const float *A,
                        const void *B, const void *C, const float *D, int chunk, float *y, float *final_state,
                        void *workspace, size_t workspace_bytes, ssd_stream_t stream) {
-  return prefill_impl(dims, dtype, x, dt, A, B, C, D, chunk, y, final_state, workspace, workspace_bytes, stream,
-                      nullptr, 0, false);
+  return prefill_impl(dims, dtype, x, dt, A, B, C, D, chunk, nullptr, y, final_state, nullptr, workspace,
+                      workspace_bytes, stream, nullptr, 0, false);
+}
+
+ssd_status ssd_prefill_ex(const ssd_dims *dims, ssd_dtype dtype, const void *x, const float *dt, const float *A,
+                          const void *B, const void *C, const float *D, int chunk, const float *initial_state,
+                          float *y, float *final_state, float *chunk_states, void *workspace, size_t workspace_bytes,
+                          ssd_stream_t stream) {
+  return prefill_impl(dims, dtype, x, dt, A, B, C, D, chunk, initial_state, y, final_state, chunk_states, workspace,
+                      workspace_bytes, stream, nullptr, 0, false);
 }
 
 ssd_status ssd_prefill_timed(const ssd_dims *dims, ssd_dtype dtype, const void *x, const float *dt, const float *A,
                              const void *B, const void *C, const float *D, int chunk, float *y, float *final_state,
                              void *workspace, size_t workspace_bytes, ssd_stream_t stream, void *const *events,
                              int num_events) {
-  return prefill_impl(dims, dtype, x, dt, A, B, C, D, chunk, y, final_state, workspace, workspace_bytes, stream,
-                      events, num_events, true);
+  return prefill_impl(dims, dtype, x, dt, A, B, C, D, chunk, nullptr, y, final_state, nullptr, workspace,
+                      workspace_bytes, stream, events, num_events, true);
 }
 
 const char *ssd_prefill_kernel_name(const ssd_dims *dims, ssd_dtype dtype, int chunk, int i) {
@@ -271,8 +288,8 @@ ssd_status prefill_into_workspace(const ssd_dims *dims, ssd_dtype dtype, const v
                                   const float *A, const void *B, const void *C, const float *D, int chunk,
                                   float *y, float *final_state, void *workspace, size_t workspace_bytes,
                                   ssd_stream_t stream) {
-  return prefill_impl(dims, dtype, x, dt, A, B, C, D, chunk, y, final_state, workspace, workspace_bytes, stream,
-                      nullptr, 0, false);
+  return prefill_impl(dims, dtype, x, dt, A, B, C, D, chunk, nullptr, y, final_state, nullptr, workspace,
+                      workspace_bytes, stream, nullptr, 0, false);
 }
 
 }  // namespace ssd

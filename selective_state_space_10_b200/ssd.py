@@ -32,7 +32,7 @@ class Dims(ctypes.Structure):
 
 # Every symbol include/ssd.h declares.
 EXPORTS = ("ssd_status_string", "ssd_version", "ssd_prefill_workspace_size",
-           "ssd_prefill_kernel_launches", "ssd_prefill", "ssd_prefill_timed",
+           "ssd_prefill_kernel_launches", "ssd_prefill", "ssd_prefill_ex", "ssd_prefill_timed",
            "ssd_prefill_kernel_name", "ssd_prefill_device_status", "ssd_prefill_noalloc",
            "ssd_prefill_noalloc_max_workspace", "ssd_decode_step")
 
@@ -54,6 +54,8 @@ def _load():
     lib.ssd_prefill_kernel_launches.restype = ci
     lib.ssd_prefill.argtypes = [dp, ci, vp, fp, fp, vp, vp, fp, ci, fp, fp, vp, sz, vp]
     lib.ssd_prefill.restype = ci
+    lib.ssd_prefill_ex.argtypes = [dp, ci, vp, fp, fp, vp, vp, fp, ci, fp, fp, fp, fp, vp, sz, vp]
+    lib.ssd_prefill_ex.restype = ci
     lib.ssd_prefill_timed.argtypes = [dp, ci, vp, fp, fp, vp, vp, fp, ci, fp, fp, vp, sz, vp,
                                       ctypes.POINTER(ctypes.c_void_p), ci]
     lib.ssd_prefill_timed.restype = ci
@@ -126,14 +128,20 @@ def _check(t: torch.Tensor, name: str, shape, dtype, device):
 
 
 def prefill(x, dt, A, B, C, D, chunk: int = 256, y=None, final_state=None, workspace=None,
-            stream=None, events=None) -> Tuple[torch.Tensor, torch.Tensor]:
-    """Chunked prefill from a zero state.  Returns (y fp32 [b,L,H,P], final_state fp32
-    [b,H,P,N]).  x, B, C are fp32 or bf16 (the same dtype); dt, A, D are fp32.
+            stream=None, events=None, initial_state=None, chunk_states=None):
+    """Chunked prefill.  Returns (y fp32 [b,L,H,P], final_state fp32 [b,H,P,N]).
+    x, B, C are fp32 or bf16 (the same dtype); dt, A, D are fp32.
+
+    `initial_state` (fp32 [b,H,P,N], optional): the state before the first token (zero if
+    None); it may be `final_state` itself.  `chunk_states`: None, True (allocate), or an
+    fp32 tensor [b, ceil(L/chunk), H, P, N] that receives the state after every chunk;
+    when given, the return value is (y, final_state, chunk_states).  Either one routes the
+    call through ssd_prefill_ex.
 
     `events`: optional list of torch.cuda.Event(enable_timing=True), at least
     prefill_kernel_launches() + 1 of them, already recorded once (so their handles
     exist); the call then goes through ssd_prefill_timed, which records events[i] before
-    kernel i and events[-1] after the last kernel."""
+    kernel i and events[-1] after the last kernel (not with initial_state/chunk_states)."""
     if x.dim() != 4 or B.dim() != 4:
         raise ValueError("x must be [b,L,H,P] and B, C [b,L,G,N]")
     if x.dtype not in _DTYPES:
@@ -155,12 +163,31 @@ def prefill(x, dt, A, B, C, D, chunk: int = 256, y=None, final_state=None, works
         final_state = torch.empty((b, H, P, N), dtype=torch.float32, device=dev)
     _check(y, "y", (b, L, H, P), torch.float32, dev)
     _check(final_state, "final_state", (b, H, P, N), torch.float32, dev)
+    if initial_state is not None:
+        _check(initial_state, "initial_state", (b, H, P, N), torch.float32, dev)
+    want_cs = chunk_states is not None and chunk_states is not False
+    if chunk_states is True:
+        chunk_states = torch.empty((b, -(-L // int(chunk)) if chunk > 0 else 0, H, P, N), dtype=torch.float32,
+                                   device=dev)
+    if want_cs:
+        _check(chunk_states, "chunk_states", (b, -(-L // int(chunk)) if chunk > 0 else 0, H, P, N),
+               torch.float32, dev)
+    extended = initial_state is not None or want_cs
+    if extended and events is not None:
+        raise ValueError("events cannot be combined with initial_state or chunk_states")
     dims = dims_of_prefill(x, B)
     dtype = _DTYPES[x.dtype]
     need = prefill_workspace_size(dims, dtype, chunk)
     if workspace is None and need > 0:
         workspace = torch.empty(need, dtype=torch.uint8, device=dev)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    if extended:
+        st = lib.ssd_prefill_ex(ctypes.byref(dims), dtype, _ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
+                                int(chunk), _ptr(initial_state), _ptr(y), _ptr(final_state),
+                                _ptr(chunk_states if want_cs else None), _ptr(workspace), ws_bytes, _stream(stream))
+        if st != OK:
+            raise SSDError(st, "ssd_prefill_ex")
+        return (y, final_state, chunk_states) if want_cs else (y, final_state)
     args = (ctypes.byref(dims), dtype, _ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
             int(chunk), _ptr(y), _ptr(final_state), _ptr(workspace), ws_bytes, _stream(stream))
     if events is None:

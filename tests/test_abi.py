@@ -160,3 +160,30 @@ def test_noalloc_validation_without_a_gpu(ssd):
     assert ssd.prefill_workspace_size(big, 1, 256) > ssd.prefill_noalloc_max_workspace()
     assert f(ctypes.byref(big), 1, v, v, v, v, v, v, 256, v, v, None) == ssd.ERR_WORKSPACE
     assert f(ctypes.byref(_dims(ssd)), 1, v, v, v, v, v, v, 48, v, v, None) == ssd.ERR_INVALID_ARG
+
+
+def _prefill_ex(ssd, dims, init=None, cs=None, ptrs=None, chunk=256):
+    p = dict(x=FAKE, dt=FAKE, A=FAKE, B=FAKE, C=FAKE, D=FAKE, y=FAKE, fs=FAKE)
+    p.update(ptrs or {})
+    v = lambda a: ctypes.c_void_p(a) if a is not None else None
+    return ssd.lib.ssd_prefill_ex(ctypes.byref(dims), 1, v(p["x"]), v(p["dt"]), v(p["A"]), v(p["B"]), v(p["C"]),
+                                  v(p["D"]), chunk, v(init), v(p["y"]), v(p["fs"]), v(cs), ctypes.c_void_p(FAKE),
+                                  1 << 40, None)
+
+
+@pytest.mark.parametrize("case", [
+    dict(init=FAKE + 4), dict(init=FAKE + 8), dict(cs=FAKE + 4), dict(cs=FAKE + 12),
+    dict(ptrs=dict(x=None)), dict(ptrs=dict(fs=FAKE + 8)), dict(chunk=48),
+])
+def test_prefill_ex_rejects_invalid(ssd, case):
+    """ssd_prefill_ex validates as ssd_prefill does, plus the optional arrays' alignment."""
+    st = _prefill_ex(ssd, _dims(ssd), init=case.get("init"), cs=case.get("cs"), ptrs=case.get("ptrs"),
+                     chunk=case.get("chunk", 256))
+    assert st == ssd.ERR_INVALID_ARG, ssd.status_string(st)
+
+
+def test_prefill_ex_empty_batch_is_a_no_op(ssd):
+    null = {k: None for k in ("x", "dt", "A", "B", "C", "D", "y", "fs")}
+    d = _dims(ssd, b=0)
+    assert ssd.lib.ssd_prefill_ex(ctypes.byref(d), 1, None, None, None, None, None, None, 256, None, None, None,
+                                  None, None, 0, None) == ssd.OK

@@ -230,3 +230,73 @@ def test_batched_decode_workload(ssd):
     for (bi, h) in pairs:
         assert_close(st[bi, h], st_ref[(bi, h)][0, 0], 2e-2, f"final state (b={bi}, h={h})")
     print(f"batched decode: worst y err {worst:.2e}")
+
+
+# ----------------------------------------------------------------- initial state, chunk states
+
+def _random_state(si, seed):
+    b, _, H, P = si.x.shape
+    N = si.B.shape[3]
+    return np.random.default_rng(seed).standard_normal((b, H, P, N)) * 0.1
+
+
+@pytest.mark.parametrize("dtype,shape", [
+    ("bf16", dict(b=2, L=600, H=4, P=64, N=128, G=1, Q=256)),   # tensor-core path, ragged tail
+    ("bf16", dict(b=1, L=300, H=4, P=64, N=128, G=2, Q=128)),   # tensor-core path, two groups
+    ("f32", dict(b=2, L=200, H=3, P=32, N=64, G=1, Q=64)),      # CUDA-core path
+    ("bf16", dict(b=1, L=100, H=2, P=16, N=32, G=1, Q=32)),     # CUDA-core path, bf16 inputs
+])
+def test_prefill_from_initial_state(ssd, dtype, shape):
+    """Prefill from a non-zero state equals the recurrence started from that state; the
+    state after every chunk equals the recurrence's state at that chunk's last token."""
+    s = shape
+    si = inputs.sequence(s["b"], s["L"], s["H"], s["P"], s["N"], s["G"], dtype, seed=321)
+    h0 = _random_state(si, 5)
+    t = to_device(si)
+    init = torch.from_numpy(h0.astype(np.float32)).cuda()
+    y, fs, cs = ssd.prefill(t["x"], t["dt"], t["A"], t["B"], t["C"], t["D"], chunk=s["Q"], initial_state=init,
+                            chunk_states=True)
+    torch.cuda.synchronize()
+    y_ref, fs_ref = oracle.recurrence(si.x, si.dt, si.A, si.B, si.C, si.D, state=h0)
+    tol = TOL[dtype]
+    assert_close(y.cpu().numpy(), y_ref, tol, "y from an initial state")
+    assert_close(fs.cpu().numpy(), fs_ref, tol, "final state from an initial state")
+    cs = cs.cpu().numpy()
+    nc = -(-s["L"] // s["Q"])
+    assert cs.shape == (s["b"], nc, s["H"], s["P"], s["N"])
+    for c in range(nc):
+        end = min((c + 1) * s["Q"], s["L"])
+        pre = si.token_slice(0, end)
+        _, st_ref = oracle.recurrence(pre.x, pre.dt, pre.A, pre.B, pre.C, pre.D, state=h0)
+        assert_close(cs[:, c], st_ref, tol, f"state after chunk {c}")
+    assert np.array_equal(cs[:, -1], fs.cpu().numpy())
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_prefill_in_pieces_equals_one_prefill(ssd, dtype):
+    """Chunked continuation: prefill of 300 tokens, then of the next 220 from its final
+    state (updated in place), matches the recurrence over all 520 tokens."""
+    P, N, Q = (64, 128, 256) if dtype == "bf16" else (16, 32, 64)
+    full = inputs.sequence(2, 520, 4, P, N, 1, dtype, seed=77)
+    a, b = full.token_slice(0, 300), full.token_slice(300, 520)
+    ta, tb = to_device(a), to_device(b)
+    ya, state = ssd.prefill(ta["x"], ta["dt"], ta["A"], ta["B"], ta["C"], ta["D"], chunk=Q)
+    yb, state2 = ssd.prefill(tb["x"], tb["dt"], tb["A"], tb["B"], tb["C"], tb["D"], chunk=Q, initial_state=state,
+                             final_state=state)
+    torch.cuda.synchronize()
+    assert state2.data_ptr() == state.data_ptr()
+    y_ref, fs_ref = oracle.recurrence(full.x, full.dt, full.A, full.B, full.C, full.D)
+    tol = TOL[dtype]
+    assert_close(np.concatenate([ya.cpu().numpy(), yb.cpu().numpy()], axis=1), y_ref, tol, "y over both pieces")
+    assert_close(state.cpu().numpy(), fs_ref, tol, "state after both pieces")
+
+
+def test_prefill_ex_without_tokens_copies_the_state(ssd):
+    si = inputs.sequence(1, 0, 2, 64, 128, 1, "bf16", seed=3)
+    t = to_device(si)
+    h0 = torch.randn(1, 2, 64, 128, device="cuda")
+    y, fs, cs = ssd.prefill(t["x"], t["dt"], t["A"], t["B"], t["C"], t["D"], chunk=256, initial_state=h0,
+                            chunk_states=True)
+    torch.cuda.synchronize()
+    assert cs.shape[1] == 0
+    assert torch.equal(fs, h0)
