@@ -500,6 +500,54 @@ def decode_leg(args, dev, rank, world, peaks, sampler):
     sampler.active(False)
     graph_ms = max_over_ranks(a.elapsed_time(e), world, dev)
     del g
+    # (3) windowed (ReplaySSM-style) decode of the same steps: the state read every step,
+    # written once per window of W tokens
+    Wn = 16
+    bufs = ssd.window_buffers(state, Wn, dtype=torch.bfloat16, ngroups=G)
+    def wstep(k):
+        ssd.decode_window_step(state, bufs, k % Wn, xs[k], dts[k], A, Bs[k], Cs[k], D, y=y, stream=stream)
+        if k % Wn == Wn - 1:
+            ssd.decode_window_flush(state, bufs, Wn, A, stream=stream)
+    for k in range(Wn):
+        wstep(k)
+    torch.cuda.synchronize(dev)
+    nw = nsteps - nsteps % Wn
+    barrier(world, dev)
+    torch.cuda.synchronize(dev)
+    sampler.active(True)
+    a, e = mk(), mk()
+    a.record(stream)
+    for k in range(nw):
+        wstep(k)
+    e.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world, dev)
+    sampler.active(False)
+    win_plain_ms = max_over_ranks(a.elapsed_time(e), world, dev)
+    # the same windowed steps from a CUDA graph (host launch overhead removed)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(cap):
+        with torch.cuda.graph(g, stream=cap):
+            for k in range(nw):
+                ssd.decode_window_step(state, bufs, k % Wn, xs[k], dts[k], A, Bs[k], Cs[k], D, y=y, stream=cap)
+                if k % Wn == Wn - 1:
+                    ssd.decode_window_flush(state, bufs, Wn, A, stream=cap)
+    torch.cuda.synchronize(dev)
+    g.replay()
+    torch.cuda.synchronize(dev)
+    barrier(world, dev)
+    torch.cuda.synchronize(dev)
+    sampler.active(True)
+    a, e = mk(), mk()
+    a.record(stream)
+    g.replay()
+    e.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world, dev)
+    sampler.active(False)
+    win_graph_ms = max_over_ranks(a.elapsed_time(e), world, dev)
+    del g
+    win_ms = min(win_plain_ms, win_graph_ms)
     state_bytes = b * H * P * N * 4
     step_bytes = 2 * state_bytes + b * H * P * (2 + 4) + b * H * 4 + 2 * b * G * N * 2 + 2 * H * 4
     best_ms = min(plain_ms, graph_ms) / nsteps
@@ -515,6 +563,15 @@ def decode_leg(args, dev, rank, world, peaks, sampler):
                      "peak_source": f"{peaks['source']} hbm_gbs",
                      "duration": "per-launch average over back-to-back launches (CUDA graph replay if faster)"},
         "gpu_launches": nsteps,
+        "windowed": {"window": Wn, "steps": nw, "value": world * nw / (win_ms / 1e3), "unit": "steps/s",
+                     "ms_per_step": win_ms / nw, "plain_ms_per_step": win_plain_ms / nw,
+                     "graph_ms_per_step": win_graph_ms / nw,
+                     "speedup_vs_standard_step": (min(plain_ms, graph_ms) / nsteps)
+                     / (win_ms / nw),
+                     "state_bytes_per_step": state_bytes * (1 + 2.0 / Wn),
+                     "state_GB/s": state_bytes * (1 + 2.0 / Wn) / (win_ms / nw / 1e3) / 1e9,
+                     "note": "per step the state is read once; every W steps one flush reads and writes it "
+                             "(ReplaySSM, SketchSSM Table 4: read D, write D/W)"},
         "config": {"workload": w.name, "batch": b, "nheads": H, "headdim": P, "dstate": N, "ngroups": G,
                    "input_dtype": "bf16", "state_dtype": "f32", "y_dtype": "f32",
                    "l2": "state (671 MB) larger than L2; no flush"},
@@ -550,6 +607,74 @@ def decode_leg(args, dev, rank, world, peaks, sampler):
     return res
 
 
+def decode_vs_recompute_leg(dev, context=4096):
+    """The cost of one new token two ways, with libssd's own calls ("Compiler-First State
+    Space Duality ..." abstract compares cached decode with full-prefix recomputation at a
+    4096-token context): one cached ssd_decode_step from the prefill's final state, against
+    an ssd_prefill of the whole context plus the new token.  Batch 1, bf16 inputs, both
+    timed back to back on one stream (the decode state, 0.8-2.6 MB, stays in L2 as in a
+    decode loop).  Also checks that both give the new token the same output."""
+    import torch
+    from selective_state_space_10_b200 import inputs, ssd
+    stream = torch.cuda.current_stream(dev)
+    mk = lambda: torch.cuda.Event(enable_timing=True)
+    out = {"context": context, "batch": 1, "chunk": 256,
+           "pages": "27-36x faster cached decode than full-prefix recompute (full models, TPU v6e)"}
+    for name, H in (("mamba2_130m", 24), ("mamba2_2.7b", 80)):
+        si = inputs.sequence(1, context + 1, H, 64, 128, 1, "bf16", seed=20261000 + H)
+        t = upload(si, dev)
+        ctx = {k: (v[:, :context].contiguous() if v.dim() > 1 else v) for k, v in t.items()}
+        tok = {"x": t["x"][:, context].contiguous(), "dt": t["dt"][:, context].contiguous(), "A": t["A"],
+               "B": t["B"][:, context].contiguous(), "C": t["C"][:, context].contiguous(), "D": t["D"]}
+        _, cache = ssd.prefill(**ctx, chunk=256)
+        state = cache.clone()
+        y_dec = ssd.decode_step(state, **tok)
+        y_full, _ = ssd.prefill(**t, chunk=256)
+        torch.cuda.synchronize(dev)
+        ref = y_full[:, context]
+        rms = float(ref.pow(2).mean().sqrt())
+        agree = float((y_dec - ref).abs().max()) / max(rms, 1e-30)
+        y = torch.empty_like(y_dec)
+        ws = torch.empty(ssd.prefill_workspace_size(ssd.dims_of_prefill(t["x"], t["B"]), ssd.BF16, 256),
+                         dtype=torch.uint8, device=dev)
+        yf = torch.empty_like(y_full)
+        fs = torch.empty_like(cache)
+        nd, nr = 200, 20
+        for _ in range(10):
+            ssd.decode_step(state, **tok, y=y, stream=stream)
+        # the decode steps are replayed from a CUDA graph, as a decode loop would, so that
+        # host launch overhead does not stand in for the step's device time
+        g = torch.cuda.CUDAGraph()
+        cap = torch.cuda.Stream(dev)
+        cap.wait_stream(stream)
+        with torch.cuda.stream(cap):
+            with torch.cuda.graph(g, stream=cap):
+                for _ in range(nd):
+                    ssd.decode_step(state, **tok, y=y, stream=cap)
+        torch.cuda.synchronize(dev)
+        g.replay()
+        torch.cuda.synchronize(dev)
+        a, e = mk(), mk()
+        a.record(stream)
+        g.replay()
+        e.record(stream)
+        torch.cuda.synchronize(dev)
+        del g
+        dec_us = a.elapsed_time(e) * 1e3 / nd
+        for _ in range(3):
+            ssd.prefill(**t, chunk=256, y=yf, final_state=fs, workspace=ws, stream=stream)
+        a, e = mk(), mk()
+        a.record(stream)
+        for _ in range(nr):
+            ssd.prefill(**t, chunk=256, y=yf, final_state=fs, workspace=ws, stream=stream)
+        e.record(stream)
+        torch.cuda.synchronize(dev)
+        rec_us = a.elapsed_time(e) * 1e3 / nr
+        out[name] = {"nheads": H, "decode_us": dec_us, "recompute_us": rec_us, "ratio": rec_us / dec_us,
+                     "new_token_output_agreement_max_over_rms": agree}
+    return out
+
+
 def run_ours(args):
     import torch
     rank, world, local = dist_env()
@@ -569,6 +694,7 @@ def run_ours(args):
     try:
         pre = prefill_leg(args, dev, rank, world, peaks, sampler)
         dec = None if args.skip_decode else decode_leg(args, dev, rank, world, peaks, sampler)
+        dvr = None if args.skip_recompute else decode_vs_recompute_leg(dev)
     finally:
         sampler.stop()
     from selective_state_space_10_b200 import inputs
@@ -584,6 +710,8 @@ def run_ours(args):
     }
     if dec:
         out["decode"] = dec
+    if dvr:
+        out["decode_vs_recompute"] = dvr
     if rank == 0 and world == 1 and not args.skip_cpu_baseline:
         w = inputs.BY_NAME[args.workload]
         rate, desc, threads, secs = oracle_prefill_rate(w, w.seed)
@@ -648,6 +776,8 @@ def main(argv=None):
     ap.add_argument("--decode-steps", type=int, default=1024)
     ap.add_argument("--skip-decode", action="store_true")
     ap.add_argument("--skip-cpu-baseline", action="store_true")
+    ap.add_argument("--skip-recompute", action="store_true",
+                    help="skip the cached-decode vs full-prefix-recompute comparison")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

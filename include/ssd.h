@@ -228,6 +228,38 @@ SSD_API ssd_status ssd_decode_step(const ssd_dims *dims, ssd_dtype dtype, float 
                            const float *dt, const float *A, const void *B, const void *C,
                            const float *D, float *y, ssd_stream_t stream);
 
+/*
+ * Windowed cached decode: ReplaySSM as "SketchSSM: Write to the Full State, Read from a
+ * Compact Sketch" summarises it (abstract; Table 4: per state head per decode step, read
+ * D and write D/W, against read D + write D for ssd_decode_step).  The state is read at
+ * every step but written only when a window of up to `window` buffered tokens is folded
+ * into it.  The outputs and the state after a flush are those of ssd_decode_step over
+ * the same tokens (the same recurrence, unrolled over the window).
+ *
+ * Window buffers, caller-owned device arrays of the call's dtype (fp32 for win_dt):
+ *   win_x [batch, window, nheads, headdim], win_dt [batch, window, nheads],
+ *   win_B [batch, window, ngroups, dstate];  contents are managed by these two calls.
+ *
+ * ssd_decode_window_step: one token, with `pos` tokens (0 .. window-1) already buffered
+ * since the state was last flushed.  Reads `state` (the committed state, not modified),
+ * writes y (this token's output) and stores the token in buffer slot `pos`.  x, dt, B, C,
+ * D, y as for ssd_decode_step.  The caller then calls ssd_decode_window_flush once the
+ * window is full (pos + 1 == window), or earlier.
+ *
+ * ssd_decode_window_flush: folds the first `count` (0 .. window) buffered tokens into
+ * `state` in place (one read and one write per head); the next window starts at pos 0.
+ *
+ * window: 1 .. 16.  Errors: as ssd_decode_step, plus SSD_ERR_INVALID_ARG for a window,
+ * pos or count out of range or a misaligned buffer (win_x, win_B 16-byte, win_dt 4-byte).
+ */
+SSD_API ssd_status ssd_decode_window_step(const ssd_dims *dims, ssd_dtype dtype, int window, int pos,
+                                          const float *state, void *win_x, float *win_dt, void *win_B,
+                                          const void *x, const float *dt, const float *A, const void *B,
+                                          const void *C, const float *D, float *y, ssd_stream_t stream);
+SSD_API ssd_status ssd_decode_window_flush(const ssd_dims *dims, ssd_dtype dtype, int window, int count,
+                                           float *state, const void *win_x, const float *win_dt,
+                                           const void *win_B, const float *A, ssd_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

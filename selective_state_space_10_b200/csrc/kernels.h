@@ -38,4 +38,13 @@ template <typename T>
 cudaError_t launch_decode_step(float *state, const T *x, const float *dt, const float *A, const T *B,
                                const T *C, const float *D, float *y, const Dims &d, cudaStream_t st);
 
+// decode_window.cu (window length 1 .. 16)
+template <typename T>
+cudaError_t launch_decode_window_step(const float *state, T *win_x, float *win_dt, T *win_B, int W, int pos,
+                                      const T *x, const float *dt, const float *A, const T *B, const T *C,
+                                      const float *D, float *y, const Dims &d, cudaStream_t st);
+template <typename T>
+cudaError_t launch_decode_window_flush(float *state, const T *win_x, const float *win_dt, const T *win_B, int W,
+                                       int count, const float *A, const Dims &d, cudaStream_t st);
+
 }  // namespace ssd

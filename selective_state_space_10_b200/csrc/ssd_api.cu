@@ -278,6 +278,57 @@ ssd_status ssd_decode_step(const ssd_dims *dims, ssd_dtype dtype, float *state, 
       static_cast<const __nv_bfloat16 *>(C), D, y, d, st));
 }
 
+ssd_status ssd_decode_window_step(const ssd_dims *dims, ssd_dtype dtype, int window, int pos, const float *state,
+                                  void *win_x, float *win_dt, void *win_B, const void *x, const float *dt,
+                                  const float *A, const void *B, const void *C, const float *D, float *y,
+                                  ssd_stream_t stream) {
+  Dims d;
+  ssd_status s = check_dims(dims, dtype, false, &d);
+  if (s != SSD_OK) return s;
+  if (window < 1 || window > 16 || pos < 0 || pos >= window) return SSD_ERR_INVALID_ARG;
+  const int64_t nx = (int64_t)d.b * d.H * d.P, nbc = (int64_t)d.b * d.G * d.N;
+  const int64_t nst = (int64_t)d.b * d.H * d.P * d.N, nh = d.b > 0 ? d.H : 0;
+  if (!check_ptr(state, nst, 16) || !check_ptr(x, nx, 16) || !check_ptr(B, nbc, 16) || !check_ptr(C, nbc, 16) ||
+      !check_ptr(y, nx, 16) || !check_ptr(dt, (int64_t)d.b * d.H, 4) || !check_ptr(A, nh, 4) ||
+      !check_ptr(D, nh, 4) || !check_ptr(win_x, nx * window, 16) || !check_ptr(win_dt, (int64_t)d.b * d.H * window, 4) ||
+      !check_ptr(win_B, nbc * window, 16))
+    return SSD_ERR_INVALID_ARG;
+  if (d.b == 0) return SSD_OK;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (dtype == SSD_F32)
+    return cuda_status(ssd::launch_decode_window_step<float>(
+        state, static_cast<float *>(win_x), win_dt, static_cast<float *>(win_B), window, pos,
+        static_cast<const float *>(x), dt, A, static_cast<const float *>(B), static_cast<const float *>(C), D, y, d,
+        st));
+  return cuda_status(ssd::launch_decode_window_step<__nv_bfloat16>(
+      state, static_cast<__nv_bfloat16 *>(win_x), win_dt, static_cast<__nv_bfloat16 *>(win_B), window, pos,
+      static_cast<const __nv_bfloat16 *>(x), dt, A, static_cast<const __nv_bfloat16 *>(B),
+      static_cast<const __nv_bfloat16 *>(C), D, y, d, st));
+}
+
+ssd_status ssd_decode_window_flush(const ssd_dims *dims, ssd_dtype dtype, int window, int count, float *state,
+                                   const void *win_x, const float *win_dt, const void *win_B, const float *A,
+                                   ssd_stream_t stream) {
+  Dims d;
+  ssd_status s = check_dims(dims, dtype, false, &d);
+  if (s != SSD_OK) return s;
+  if (window < 1 || window > 16 || count < 0 || count > window) return SSD_ERR_INVALID_ARG;
+  const int64_t nx = (int64_t)d.b * d.H * d.P, nbc = (int64_t)d.b * d.G * d.N;
+  const int64_t nst = (int64_t)d.b * d.H * d.P * d.N, nh = d.b > 0 ? d.H : 0;
+  if (!check_ptr(state, nst, 16) || !check_ptr(A, nh, 4) || !check_ptr(win_x, nx * window, 16) ||
+      !check_ptr(win_dt, (int64_t)d.b * d.H * window, 4) || !check_ptr(win_B, nbc * window, 16))
+    return SSD_ERR_INVALID_ARG;
+  if (d.b == 0 || count == 0) return SSD_OK;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (dtype == SSD_F32)
+    return cuda_status(ssd::launch_decode_window_flush<float>(state, static_cast<const float *>(win_x), win_dt,
+                                                              static_cast<const float *>(win_B), window, count, A,
+                                                              d, st));
+  return cuda_status(ssd::launch_decode_window_flush<__nv_bfloat16>(
+      state, static_cast<const __nv_bfloat16 *>(win_x), win_dt, static_cast<const __nv_bfloat16 *>(win_B), window,
+      count, A, d, st));
+}
+
 }  // extern "C"
 
 namespace ssd {

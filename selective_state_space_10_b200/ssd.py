@@ -34,7 +34,8 @@ class Dims(ctypes.Structure):
 EXPORTS = ("ssd_status_string", "ssd_version", "ssd_prefill_workspace_size",
            "ssd_prefill_kernel_launches", "ssd_prefill", "ssd_prefill_ex", "ssd_prefill_timed",
            "ssd_prefill_kernel_name", "ssd_prefill_device_status", "ssd_prefill_noalloc",
-           "ssd_prefill_noalloc_max_workspace", "ssd_decode_step")
+           "ssd_prefill_noalloc_max_workspace", "ssd_decode_step", "ssd_decode_window_step",
+           "ssd_decode_window_flush")
 
 
 def _load():
@@ -69,6 +70,10 @@ def _load():
     lib.ssd_prefill_noalloc_max_workspace.restype = sz
     lib.ssd_decode_step.argtypes = [dp, ci, fp, vp, fp, fp, vp, vp, fp, fp, vp]
     lib.ssd_decode_step.restype = ci
+    lib.ssd_decode_window_step.argtypes = [dp, ci, ci, ci, fp, vp, fp, vp, vp, fp, fp, vp, vp, fp, fp, vp]
+    lib.ssd_decode_window_step.restype = ci
+    lib.ssd_decode_window_flush.argtypes = [dp, ci, ci, ci, fp, vp, fp, vp, fp, vp]
+    lib.ssd_decode_window_flush.restype = ci
     return lib
 
 
@@ -284,3 +289,57 @@ def prefill_host(x, dt, A, B, C, D, chunk: int = 256, device="cuda", stream=None
         y_h.copy_(y, non_blocking=True)
         fs_h.copy_(fs, non_blocking=True)
     return y_h, fs_h
+
+
+def window_buffers(state: torch.Tensor, window: int, dtype=torch.bfloat16, ngroups: int = 1):
+    """Device buffers for the windowed decode of a state [b,H,P,N]: (win_x [b,W,H,P],
+    win_dt [b,W,H] fp32, win_B [b,W,G,N]), in the call's input dtype."""
+    b, H, P, N = state.shape
+    dev = state.device
+    return (torch.empty((b, window, H, P), dtype=dtype, device=dev),
+            torch.empty((b, window, H), dtype=torch.float32, device=dev),
+            torch.empty((b, window, ngroups, N), dtype=dtype, device=dev))
+
+
+def decode_window_step(state, buffers, pos: int, x, dt, A, B, C, D, y=None, stream=None) -> torch.Tensor:
+    """ssd_decode_window_step: this token's y from the committed `state` (not modified) and
+    the `pos` tokens buffered since the last flush; stores the token in slot `pos`."""
+    win_x, win_dt, win_B = buffers
+    b, H, P, N = state.shape
+    G = B.shape[1]
+    dev = state.device
+    if x.dtype not in _DTYPES:
+        raise ValueError(f"unsupported input dtype {x.dtype}")
+    W = win_x.shape[1]
+    _check(state, "state", (b, H, P, N), torch.float32, dev)
+    _check(win_x, "win_x", (b, W, H, P), x.dtype, dev)
+    _check(win_dt, "win_dt", (b, W, H), torch.float32, dev)
+    _check(win_B, "win_B", (b, W, G, N), x.dtype, dev)
+    for name, t, shape, dtype in (("x", x, (b, H, P), x.dtype), ("dt", dt, (b, H), torch.float32),
+                                  ("A", A, (H,), torch.float32), ("B", B, (b, G, N), x.dtype),
+                                  ("C", C, (b, G, N), x.dtype), ("D", D, (H,), torch.float32)):
+        _check(t, name, shape, dtype, dev)
+    if y is None:
+        y = torch.empty((b, H, P), dtype=torch.float32, device=dev)
+    _check(y, "y", (b, H, P), torch.float32, dev)
+    st = lib.ssd_decode_window_step(ctypes.byref(_dims(b, 1, H, P, N, G)), _DTYPES[x.dtype], W, int(pos),
+                                    _ptr(state), _ptr(win_x), _ptr(win_dt), _ptr(win_B), _ptr(x), _ptr(dt),
+                                    _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(y), _stream(stream))
+    if st != OK:
+        raise SSDError(st, "ssd_decode_window_step")
+    return y
+
+
+def decode_window_flush(state, buffers, count: int, A, stream=None) -> torch.Tensor:
+    """ssd_decode_window_flush: folds the first `count` buffered tokens into `state`."""
+    win_x, win_dt, win_B = buffers
+    b, H, P, N = state.shape
+    W, G = win_x.shape[1], win_B.shape[2]
+    if win_x.dtype not in _DTYPES:
+        raise ValueError(f"unsupported input dtype {win_x.dtype}")
+    st = lib.ssd_decode_window_flush(ctypes.byref(_dims(b, 1, H, P, N, G)), _DTYPES[win_x.dtype], W, int(count),
+                                     _ptr(state), _ptr(win_x), _ptr(win_dt), _ptr(win_B), _ptr(A),
+                                     _stream(stream))
+    if st != OK:
+        raise SSDError(st, "ssd_decode_window_flush")
+    return state

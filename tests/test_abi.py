@@ -187,3 +187,17 @@ def test_prefill_ex_empty_batch_is_a_no_op(ssd):
     d = _dims(ssd, b=0)
     assert ssd.lib.ssd_prefill_ex(ctypes.byref(d), 1, None, None, None, None, None, None, 256, None, None, None,
                                   None, None, 0, None) == ssd.OK
+
+
+def test_window_decode_rejects_invalid(ssd):
+    """Window, position and count ranges and buffer alignment are checked on the host."""
+    d = _dims(ssd, L=1)
+    v = ctypes.c_void_p(FAKE)
+    step = lambda W, pos, wx=FAKE: ssd.lib.ssd_decode_window_step(ctypes.byref(d), 1, W, pos, v, ctypes.c_void_p(wx),
+                                                                 v, v, v, v, v, v, v, v, v, None)
+    flush = lambda W, cnt: ssd.lib.ssd_decode_window_flush(ctypes.byref(d), 1, W, cnt, v, v, v, v, v, None)
+    for W, pos in ((0, 0), (17, 0), (16, 16), (4, -1)):
+        assert step(W, pos) == ssd.ERR_INVALID_ARG
+    assert step(16, 3, FAKE + 8) == ssd.ERR_INVALID_ARG
+    for W, cnt in ((0, 0), (17, 1), (8, 9), (8, -1)):
+        assert flush(W, cnt) == ssd.ERR_INVALID_ARG

@@ -300,3 +300,42 @@ def test_prefill_ex_without_tokens_copies_the_state(ssd):
     torch.cuda.synchronize()
     assert cs.shape[1] == 0
     assert torch.equal(fs, h0)
+
+
+# ----------------------------------------------------------------- windowed decode
+
+@pytest.mark.parametrize("dtype,shape,W", [
+    ("bf16", dict(b=3, H=4, P=64, N=128, G=1), 16),
+    ("bf16", dict(b=2, H=4, P=64, N=128, G=2), 5),
+    ("f32", dict(b=2, H=3, P=32, N=64, G=1), 16),
+    ("f32", dict(b=1, H=2, P=100, N=16, G=1), 7),
+    ("bf16", dict(b=1, H=2, P=256, N=256, G=1), 1),
+])
+def test_windowed_decode_matches_the_recurrence(ssd, dtype, shape, W):
+    """ReplaySSM-style decode after a prefill: per token y from the committed state and the
+    buffered window, the state written only at flushes (every W tokens, and a partial
+    window at the end), against the fp64 recurrence over all tokens."""
+    s = shape
+    L0, K = 200, 2 * W + 3
+    full = inputs.sequence(s["b"], L0 + K, s["H"], s["P"], s["N"], s["G"], dtype, seed=99)
+    pre = full.token_slice(0, L0)
+    t = to_device(pre)
+    _, state = ssd.prefill(t["x"], t["dt"], t["A"], t["B"], t["C"], t["D"], chunk=64)
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    bufs = ssd.window_buffers(state, W, dtype=tdt, ngroups=s["G"])
+    ys, pos = [], 0
+    for k in range(K):
+        tok = decode_args(to_device(full.token_slice(L0 + k, L0 + k + 1)))
+        ys.append(ssd.decode_window_step(state, bufs, pos, **tok).cpu().numpy())
+        pos += 1
+        if pos == W:
+            ssd.decode_window_flush(state, bufs, pos, tok["A"])
+            pos = 0
+    ssd.decode_window_flush(state, bufs, pos, tok["A"])
+    torch.cuda.synchronize()
+    y_ref, st_ref = oracle.recurrence(full.x, full.dt, full.A, full.B, full.C, full.D)
+    y_w = np.stack(ys, axis=1)
+    tol = TOL[dtype]
+    for k in range(K):  # per-step bound, as for the decode workloads
+        assert_close(y_w[:, k], y_ref[:, L0 + k], tol, f"windowed y at step {k}")
+    assert_close(state.cpu().numpy(), st_ref, tol, "state after the windows")
