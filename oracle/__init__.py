@@ -9,3 +9,4 @@ from .oracle import (  # noqa: F401
     chunked,
     default_threads,
 )
+from .frontend import frontend, causal_conv, softplus, silu  # noqa: F401,E402
