@@ -229,6 +229,38 @@ SSD_API ssd_status ssd_decode_step(const ssd_dims *dims, ssd_dtype dtype, float 
                            const float *D, float *y, ssd_stream_t stream);
 
 /*
+ * The block's front end, right before the SSD layer ("Engineering Hybrid State-Space
+ * Models" section 3: a width-4 1-D convolution with SiLU, Delta = Softplus(Linear(x) +
+ * bias), and the convState of the last dConv - 1 = 3 inputs per channel), in one pass:
+ *
+ *   a[t, c]  = silu( sum_{k=0..3} conv_w[c, k] * xbc[t - 3 + k, c] + conv_b[c] )
+ *   x, B, C  = a split by channel: [0, H*P) -> x, then G*N -> B, then G*N -> C
+ *   dt[t, h] = softplus(dt_raw[t, h] + dt_bias[h]),  softplus(z) = log(1 + exp(z))
+ *
+ *   xbc            [batch, seqlen, H*P + 2*G*N] in the call's dtype (the projected
+ *                  x, B and C channels; the projection itself is the caller's)
+ *   conv_w         [H*P + 2*G*N, 4] fp32, 16-byte aligned (tap k = 3 multiplies token t)
+ *   conv_b         [H*P + 2*G*N] fp32, or NULL for no bias
+ *   conv_state_in  [batch, 3, H*P + 2*G*N] fp32: the three inputs before the first token,
+ *                  oldest first, or NULL for zeros (a new sequence)
+ *   conv_state_out same shape: receives the last three inputs (from conv_state_in too
+ *                  when seqlen < 3), or NULL; it may be conv_state_in (updated in place)
+ *   dt_raw, dt     [batch, seqlen, nheads] fp32 (dt may be dt_raw); dt_bias [nheads] fp32
+ *   x, B, C        the ssd_prefill input layouts in the call's dtype (bf16: rounded to
+ *                  nearest even from the fp32 result), 16-byte aligned
+ *
+ * With seqlen = 1 and the conv state in place this is the decode-time front end of one
+ * token (x, B, C then have ssd_decode_step's layouts).  The convolution is depthwise and
+ * causal, as the page's width-4 conv is read here.  Errors: as ssd_prefill for the
+ * dims; SSD_ERR_INVALID_ARG for NULL or misaligned arrays, and for batch > 65535 or more
+ * than 65535 * 256 channels (launch grid limits).
+ */
+SSD_API ssd_status ssd_frontend(const ssd_dims *dims, ssd_dtype dtype, const void *xbc, const float *conv_w,
+                                const float *conv_b, const float *conv_state_in, float *conv_state_out,
+                                const float *dt_raw, const float *dt_bias, void *x, void *B, void *C, float *dt,
+                                ssd_stream_t stream);
+
+/*
  * Windowed cached decode: ReplaySSM as "SketchSSM: Write to the Full State, Read from a
  * Compact Sketch" summarises it (abstract; Table 4: per state head per decode step, read
  * D and write D/W, against read D + write D for ssd_decode_step).  The state is read at

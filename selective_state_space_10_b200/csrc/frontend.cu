@@ -1,0 +1,220 @@
+// frontend.cu -- the steps of the Mamba-2 block right before the SSD layer ("Engineering
+// Hybrid State-Space Models" section 3, the block diagram: a width-4 1-D convolution and
+// SiLU; Delta = Softplus(Linear(x) + bias); the session's convState of the last dConv-1
+// inputs per channel), fused into one pass over the projected inputs:
+//
+//   u = xbc [b, L, H*P + 2*G*N]   (the x, B and C channels, in that order)
+//   a[t, c] = silu( sum_k w[c, k] u[t - 3 + k, c] + bias[c] )   (inputs before the first
+//             token from the conv state, or zero)
+//   x = a[:, :, :HP], B = a[:, :, HP:HP+GN], C = a[:, :, HP+GN:]   (the SSD layouts)
+//   dt[t, h] = softplus(dt_raw[t, h] + dt_bias[h])
+//
+// k_frontend: one thread per (4 channels, 8-token run) -- grid (token runs, channel tiles,
+// batch rows); consecutive threads take consecutive channel groups, so every vector load
+// and store of a warp is one contiguous run of the token's row, and all of a thread's
+// inputs are loaded before the first use.  fp32 arithmetic; outputs in the call's dtype
+// (round to nearest even for bf16).  The CTAs of the first channel tile
+// also form dt for their tokens.  k_frontend_state then writes the new conv state (the
+// last three inputs), after every read of the old one, so the state may be updated in
+// place.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace ssd {
+
+constexpr int kFeTokens = 8;  // tokens per thread
+
+// cp.async of 4, 8 or 16 bytes global -> shared (both addresses aligned to the size)
+template <int BYTES>
+__device__ __forceinline__ void cp_async(void *dst, const void *src) {
+  const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(dst));
+  if constexpr (BYTES == 16)
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(src) : "memory");
+  else
+    asm volatile("cp.async.ca.shared.global [%0], [%1], %2;" ::"r"(d), "l"(src), "n"(BYTES) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+template <typename T> __device__ __forceinline__ T from_f32(float v);
+template <> __device__ __forceinline__ float from_f32<float>(float v) { return v; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float v) { return __float2bfloat16_rn(v); }
+
+__device__ __forceinline__ float silu_f(float v) { return v / (1.f + __expf(-v)); }
+__device__ __forceinline__ float softplus_f(float z) { return z > 20.f ? z : log1pf(__expf(z)); }
+__device__ __forceinline__ void store_out(float *p, float v) { *p = v; }
+__device__ __forceinline__ void store_out(__nv_bfloat16 *p, float v) { *p = __float2bfloat16_rn(v); }
+
+// V consecutive channels of one token: loads and stores of V elements at once (V = 4:
+// 8 bytes of bf16 or 16 bytes of fp32), V = 1 the scalar fallback.
+template <typename T, int V> struct Vec;
+template <> struct Vec<float, 1> {
+  static __device__ __forceinline__ void load(const float *p, float (&v)[1]) { v[0] = *p; }
+  static __device__ __forceinline__ void store(float *p, const float (&v)[1]) { *p = v[0]; }
+};
+template <> struct Vec<__nv_bfloat16, 1> {
+  static __device__ __forceinline__ void load(const __nv_bfloat16 *p, float (&v)[1]) { v[0] = __bfloat162float(*p); }
+  static __device__ __forceinline__ void store(__nv_bfloat16 *p, const float (&v)[1]) { *p = __float2bfloat16_rn(v[0]); }
+};
+template <> struct Vec<float, 4> {
+  static __device__ __forceinline__ void load(const float *p, float (&v)[4]) {
+    const float4 q = *reinterpret_cast<const float4 *>(p);
+    v[0] = q.x; v[1] = q.y; v[2] = q.z; v[3] = q.w;
+  }
+  static __device__ __forceinline__ void store(float *p, const float (&v)[4]) {
+    *reinterpret_cast<float4 *>(p) = make_float4(v[0], v[1], v[2], v[3]);
+  }
+};
+template <> struct Vec<__nv_bfloat16, 4> {
+  static __device__ __forceinline__ void load(const __nv_bfloat16 *p, float (&v)[4]) {
+    const uint2 q = *reinterpret_cast<const uint2 *>(p);
+    v[0] = __uint_as_float(q.x << 16); v[1] = __uint_as_float(q.x & 0xffff0000u);
+    v[2] = __uint_as_float(q.y << 16); v[3] = __uint_as_float(q.y & 0xffff0000u);
+  }
+  static __device__ __forceinline__ void store(__nv_bfloat16 *p, const float (&v)[4]) {
+    const __nv_bfloat162 a = __floats2bfloat162_rn(v[0], v[1]), b = __floats2bfloat162_rn(v[2], v[3]);
+    uint2 q;
+    q.x = *reinterpret_cast<const uint32_t *>(&a);
+    q.y = *reinterpret_cast<const uint32_t *>(&b);
+    *reinterpret_cast<uint2 *>(p) = q;
+  }
+};
+
+// One thread per (V channels, kFeTokens-token run): grid (token runs, channel tiles of
+// 256 * V, batch rows).  V = 4 needs H * P to be a multiple of 4 (then no group of four
+// straddles the x | B | C boundaries, and every vector access is aligned).
+template <typename T, int V>
+__global__ void __launch_bounds__(256)
+k_frontend(const T *__restrict__ xbc, const float *__restrict__ w, const float *__restrict__ bias,
+           const float *__restrict__ state_in, const float *dt_raw, const float *__restrict__ dt_bias,
+           T *__restrict__ x, T *__restrict__ B, T *__restrict__ C, float *dt, Dims d) {
+  const int HP = d.H * d.P, GN = d.G * d.N, CH = HP + 2 * GN;
+  const int c = (blockIdx.y * blockDim.x + threadIdx.x) * V;
+  const int t0 = blockIdx.x * kFeTokens, bi = blockIdx.z;
+  const int t1 = min(t0 + kFeTokens, d.L);
+  if (blockIdx.y == 0) {  // dt for this run of tokens (all loads issued before any use)
+    for (int h = threadIdx.x; h < d.H; h += blockDim.x) {
+      const float bh = dt_bias[h];
+      float z[kFeTokens];
+#pragma unroll
+      for (int j = 0; j < kFeTokens; ++j)
+        z[j] = (t0 + j < t1) ? dt_raw[((size_t)bi * d.L + t0 + j) * d.H + h] : 0.f;
+#pragma unroll
+      for (int j = 0; j < kFeTokens; ++j)
+        if (t0 + j < t1) dt[((size_t)bi * d.L + t0 + j) * d.H + h] = softplus_f(z[j] + bh);
+    }
+  }
+  // Stage this CTA's inputs -- rows t0-3 .. t1-1 of its 256 * V channels -- in shared
+  // memory with asynchronous copies (nothing held in registers while they fly); rows
+  // before the sequence come from the conv state or are zero.
+  __shared__ __align__(16) T tile[3 + kFeTokens][256 * V];
+  const int tl = threadIdx.x * V;  // this thread's first channel within the tile
+  const bool active = c < CH;
+  if (active) {
+    const T *uc = xbc + (size_t)bi * d.L * CH + c;
+#pragma unroll
+    for (int j = 0; j < 3 + kFeTokens; ++j) {
+      const int t = t0 - 3 + j;
+      if (t >= 0 && t < t1) {
+        if constexpr (sizeof(T) * V >= 4)
+          cp_async<sizeof(T) * V>(&tile[j][tl], uc + (size_t)t * CH);
+        else
+          tile[j][tl] = uc[(size_t)t * CH];  // the scalar bf16 fallback (2 bytes)
+      } else if (t < 0) {
+#pragma unroll
+        for (int q = 0; q < V; ++q)
+          tile[j][tl + q] = from_f32<T>(state_in ? state_in[((size_t)bi * 3 + (3 + t)) * CH + c + q] : 0.f);
+      }
+    }
+  }
+  // the filters while the copies fly
+  float4 wc[V];
+  float bc[V];
+#pragma unroll
+  for (int q = 0; q < V; ++q) {
+    wc[q] = active ? *reinterpret_cast<const float4 *>(w + (size_t)(c + q) * 4) : make_float4(0.f, 0.f, 0.f, 0.f);
+    bc[q] = (active && bias) ? bias[c + q] : 0.f;
+  }
+  cp_async_wait_all();
+  __syncthreads();
+  if (!active) return;
+  T *dst;
+  size_t stride;
+  if (c < HP) {
+    dst = x + (size_t)bi * d.L * HP + c;
+    stride = HP;
+  } else if (c < HP + GN) {
+    dst = B + (size_t)bi * d.L * GN + (c - HP);
+    stride = GN;
+  } else {
+    dst = C + (size_t)bi * d.L * GN + (c - HP - GN);
+    stride = GN;
+  }
+  // each token from its four input rows in shared memory (a rolling window of rows)
+  float r0[V], r1[V], r2[V];
+  Vec<T, V>::load(&tile[0][tl], r0);
+  Vec<T, V>::load(&tile[1][tl], r1);
+  Vec<T, V>::load(&tile[2][tl], r2);
+#pragma unroll
+  for (int j = 0; j < kFeTokens; ++j) {
+    if (t0 + j < t1) {
+      float r3[V], o[V];
+      Vec<T, V>::load(&tile[3 + j][tl], r3);
+#pragma unroll
+      for (int q = 0; q < V; ++q) {
+        o[q] = silu_f(fmaf(wc[q].x, r0[q], fmaf(wc[q].y, r1[q], fmaf(wc[q].z, r2[q], fmaf(wc[q].w, r3[q], bc[q])))));
+        r0[q] = r1[q];
+        r1[q] = r2[q];
+        r2[q] = r3[q];
+      }
+      Vec<T, V>::store(dst + (size_t)(t0 + j) * stride, o);
+    }
+  }
+}
+
+// new_state[j, c] = input at token L - 3 + j (j = 0..2), from this call's tokens or, when
+// L < 3, from the old state; each thread reads all it needs before it writes.
+template <typename T>
+__global__ void __launch_bounds__(256)
+k_frontend_state(const T *__restrict__ xbc, const float *state_in, float *state_out, Dims d) {
+  const int CH = d.H * d.P + 2 * d.G * d.N;
+  const int c = blockIdx.x * blockDim.x + threadIdx.x, bi = blockIdx.y;
+  if (c >= CH) return;
+  float v[3];
+#pragma unroll
+  for (int j = 0; j < 3; ++j) {
+    const int t = d.L - 3 + j;
+    v[j] = t >= 0 ? to_f32(xbc[((size_t)bi * d.L + t) * CH + c])
+                  : (state_in ? state_in[((size_t)bi * 3 + (3 + t)) * CH + c] : 0.f);
+  }
+#pragma unroll
+  for (int j = 0; j < 3; ++j) state_out[((size_t)bi * 3 + j) * CH + c] = v[j];
+}
+
+template <typename T>
+cudaError_t launch_frontend(const T *xbc, const float *w, const float *bias, const float *state_in,
+                            float *state_out, const float *dt_raw, const float *dt_bias, T *x, T *B, T *C, float *dt,
+                            const Dims &d, cudaStream_t st) {
+  const int CH = d.H * d.P + 2 * d.G * d.N;
+  // token runs on x (up to 2^31 - 1), channel tiles on y and batch rows on z (the host
+  // checks both stay within 65535)
+  const unsigned runs = (unsigned)((d.L + kFeTokens - 1) / kFeTokens);
+  if ((d.H * d.P) % 4 == 0)
+    k_frontend<T, 4><<<dim3(runs, (unsigned)((CH / 4 + 255) / 256), (unsigned)d.b), 256, 0, st>>>(
+        xbc, w, bias, state_in, dt_raw, dt_bias, x, B, C, dt, d);
+  else
+    k_frontend<T, 1><<<dim3(runs, (unsigned)((CH + 255) / 256), (unsigned)d.b), 256, 0, st>>>(
+        xbc, w, bias, state_in, dt_raw, dt_bias, x, B, C, dt, d);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess || state_out == nullptr) return e;
+  k_frontend_state<T><<<dim3((unsigned)((CH + 255) / 256), (unsigned)d.b), 256, 0, st>>>(xbc, state_in, state_out, d);
+  return cudaGetLastError();
+}
+
+template cudaError_t launch_frontend<float>(const float *, const float *, const float *, const float *, float *,
+                                            const float *, const float *, float *, float *, float *, float *,
+                                            const Dims &, cudaStream_t);
+template cudaError_t launch_frontend<__nv_bfloat16>(const __nv_bfloat16 *, const float *, const float *, const float *,
+                                                    float *, const float *, const float *, __nv_bfloat16 *,
+                                                    __nv_bfloat16 *, __nv_bfloat16 *, float *, const Dims &,
+                                                    cudaStream_t);
+
+}  // namespace ssd

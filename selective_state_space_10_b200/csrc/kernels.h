@@ -38,6 +38,12 @@ template <typename T>
 cudaError_t launch_decode_step(float *state, const T *x, const float *dt, const float *A, const T *B,
                                const T *C, const float *D, float *y, const Dims &d, cudaStream_t st);
 
+// frontend.cu: conv + SiLU + split, softplus dt; the new conv state when state_out != NULL
+template <typename T>
+cudaError_t launch_frontend(const T *xbc, const float *w, const float *bias, const float *state_in,
+                            float *state_out, const float *dt_raw, const float *dt_bias, T *x, T *B, T *C, float *dt,
+                            const Dims &d, cudaStream_t st);
+
 // decode_window.cu (window length 1 .. 16)
 template <typename T>
 cudaError_t launch_decode_window_step(const float *state, T *win_x, float *win_dt, T *win_B, int W, int pos,

@@ -278,6 +278,40 @@ ssd_status ssd_decode_step(const ssd_dims *dims, ssd_dtype dtype, float *state, 
       static_cast<const __nv_bfloat16 *>(C), D, y, d, st));
 }
 
+ssd_status ssd_frontend(const ssd_dims *dims, ssd_dtype dtype, const void *xbc, const float *conv_w,
+                        const float *conv_b, const float *conv_state_in, float *conv_state_out, const float *dt_raw,
+                        const float *dt_bias, void *x, void *B, void *C, float *dt, ssd_stream_t stream) {
+  Dims d;
+  ssd_status s = check_dims(dims, dtype, true, &d);
+  if (s != SSD_OK) return s;
+  const int64_t ntok = (int64_t)d.b * d.L, ch = (int64_t)d.H * d.P + 2 * (int64_t)d.G * d.N;
+  const int64_t nx = ntok * d.H * d.P, nbc = ntok * d.G * d.N, any = ntok > 0 ? 1 : 0;
+  const size_t esz = dtype == SSD_F32 ? 4 : 2;
+  if (!check_ptr(xbc, ntok * ch, esz) || !check_ptr(conv_w, any * ch * 4, 16) || !check_ptr(x, nx, 16) ||
+      !check_ptr(B, nbc, 16) || !check_ptr(C, nbc, 16) || !check_ptr(dt_raw, ntok * d.H, 4) ||
+      !check_ptr(dt_bias, any * d.H, 4) || !check_ptr(dt, ntok * d.H, 4))
+    return SSD_ERR_INVALID_ARG;
+  if (d.b > 65535 || (ch + 255) / 256 > 65535) return SSD_ERR_INVALID_ARG;  // launch grid limits
+  const int64_t nstate = (int64_t)d.b * 3 * ch;
+  if ((conv_b != nullptr && !check_ptr(conv_b, ch, 4)) || (conv_state_in != nullptr && !check_ptr(conv_state_in, nstate, 4)) ||
+      (conv_state_out != nullptr && !check_ptr(conv_state_out, nstate, 4)))
+    return SSD_ERR_INVALID_ARG;
+  if (d.b == 0) return SSD_OK;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (d.L == 0) {  // no tokens: the conv state carries over unchanged
+    if (conv_state_out == nullptr || conv_state_out == conv_state_in) return SSD_OK;
+    if (conv_state_in == nullptr) return cuda_status(cudaMemsetAsync(conv_state_out, 0, (size_t)nstate * 4, st));
+    return cuda_status(cudaMemcpyAsync(conv_state_out, conv_state_in, (size_t)nstate * 4, cudaMemcpyDeviceToDevice, st));
+  }
+  if (dtype == SSD_F32)
+    return cuda_status(ssd::launch_frontend<float>(static_cast<const float *>(xbc), conv_w, conv_b, conv_state_in,
+                                                   conv_state_out, dt_raw, dt_bias, static_cast<float *>(x),
+                                                   static_cast<float *>(B), static_cast<float *>(C), dt, d, st));
+  return cuda_status(ssd::launch_frontend<__nv_bfloat16>(
+      static_cast<const __nv_bfloat16 *>(xbc), conv_w, conv_b, conv_state_in, conv_state_out, dt_raw, dt_bias,
+      static_cast<__nv_bfloat16 *>(x), static_cast<__nv_bfloat16 *>(B), static_cast<__nv_bfloat16 *>(C), dt, d, st));
+}
+
 ssd_status ssd_decode_window_step(const ssd_dims *dims, ssd_dtype dtype, int window, int pos, const float *state,
                                   void *win_x, float *win_dt, void *win_B, const void *x, const float *dt,
                                   const float *A, const void *B, const void *C, const float *D, float *y,

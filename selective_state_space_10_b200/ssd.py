@@ -34,7 +34,7 @@ class Dims(ctypes.Structure):
 EXPORTS = ("ssd_status_string", "ssd_version", "ssd_prefill_workspace_size",
            "ssd_prefill_kernel_launches", "ssd_prefill", "ssd_prefill_ex", "ssd_prefill_timed",
            "ssd_prefill_kernel_name", "ssd_prefill_device_status", "ssd_prefill_noalloc",
-           "ssd_prefill_noalloc_max_workspace", "ssd_decode_step", "ssd_decode_window_step",
+           "ssd_prefill_noalloc_max_workspace", "ssd_decode_step", "ssd_frontend", "ssd_decode_window_step",
            "ssd_decode_window_flush")
 
 
@@ -70,6 +70,8 @@ def _load():
     lib.ssd_prefill_noalloc_max_workspace.restype = sz
     lib.ssd_decode_step.argtypes = [dp, ci, fp, vp, fp, fp, vp, vp, fp, fp, vp]
     lib.ssd_decode_step.restype = ci
+    lib.ssd_frontend.argtypes = [dp, ci, vp, fp, fp, fp, fp, fp, fp, vp, vp, vp, fp, vp]
+    lib.ssd_frontend.restype = ci
     lib.ssd_decode_window_step.argtypes = [dp, ci, ci, ci, fp, vp, fp, vp, vp, fp, fp, vp, vp, fp, fp, vp]
     lib.ssd_decode_window_step.restype = ci
     lib.ssd_decode_window_flush.argtypes = [dp, ci, ci, ci, fp, vp, fp, vp, fp, vp]
@@ -343,3 +345,37 @@ def decode_window_flush(state, buffers, count: int, A, stream=None) -> torch.Ten
     if st != OK:
         raise SSDError(st, "ssd_decode_window_flush")
     return state
+
+
+def frontend(xbc, conv_w, dt_raw, dt_bias, nheads: int, headdim: int, ngroups: int, dstate: int, conv_b=None,
+             conv_state_in=None, conv_state_out=None, x=None, B=None, C=None, dt=None, stream=None):
+    """ssd_frontend: conv (width 4, causal, depthwise) + SiLU over xbc [b, L, H*P + 2*G*N],
+    split into x [b,L,H,P], B and C [b,L,G,N] (xbc's dtype), and dt = softplus(dt_raw +
+    dt_bias) [b,L,H] fp32.  conv_state_in / conv_state_out: fp32 [b, 3, channels] or None;
+    they may be the same tensor.  Returns (x, B, C, dt)."""
+    b, L, CH = xbc.shape
+    H, P, G, N = int(nheads), int(headdim), int(ngroups), int(dstate)
+    if CH != H * P + 2 * G * N:
+        raise ValueError(f"xbc has {CH} channels, expected {H * P + 2 * G * N}")
+    if xbc.dtype not in _DTYPES:
+        raise ValueError(f"unsupported input dtype {xbc.dtype}")
+    dev = xbc.device
+    _check(xbc, "xbc", (b, L, CH), xbc.dtype, dev)
+    _check(conv_w, "conv_w", (CH, 4), torch.float32, dev)
+    _check(dt_raw, "dt_raw", (b, L, H), torch.float32, dev)
+    _check(dt_bias, "dt_bias", (H,), torch.float32, dev)
+    if conv_b is not None:
+        _check(conv_b, "conv_b", (CH,), torch.float32, dev)
+    for name, t in (("conv_state_in", conv_state_in), ("conv_state_out", conv_state_out)):
+        if t is not None:
+            _check(t, name, (b, 3, CH), torch.float32, dev)
+    x = torch.empty((b, L, H, P), dtype=xbc.dtype, device=dev) if x is None else x
+    B = torch.empty((b, L, G, N), dtype=xbc.dtype, device=dev) if B is None else B
+    C = torch.empty((b, L, G, N), dtype=xbc.dtype, device=dev) if C is None else C
+    dt = torch.empty((b, L, H), dtype=torch.float32, device=dev) if dt is None else dt
+    st = lib.ssd_frontend(ctypes.byref(_dims(b, L, H, P, N, G)), _DTYPES[xbc.dtype], _ptr(xbc), _ptr(conv_w),
+                          _ptr(conv_b), _ptr(conv_state_in), _ptr(conv_state_out), _ptr(dt_raw), _ptr(dt_bias),
+                          _ptr(x), _ptr(B), _ptr(C), _ptr(dt), _stream(stream))
+    if st != OK:
+        raise SSDError(st, "ssd_frontend")
+    return x, B, C, dt

@@ -201,3 +201,19 @@ def test_window_decode_rejects_invalid(ssd):
     assert step(16, 3, FAKE + 8) == ssd.ERR_INVALID_ARG
     for W, cnt in ((0, 0), (17, 1), (8, 9), (8, -1)):
         assert flush(W, cnt) == ssd.ERR_INVALID_ARG
+
+
+def test_frontend_rejects_invalid(ssd):
+    """ssd_frontend validates its arrays (alignment, NULL) and grid limits on the host."""
+    v = lambda a: ctypes.c_void_p(a) if a is not None else None
+    def call(d, **over):
+        p = dict(xbc=FAKE, w=FAKE, b=None, si=None, so=None, dtr=FAKE, dtb=FAKE, x=FAKE, B=FAKE, C=FAKE, dt=FAKE)
+        p.update(over)
+        return ssd.lib.ssd_frontend(ctypes.byref(d), 1, v(p["xbc"]), v(p["w"]), v(p["b"]), v(p["si"]), v(p["so"]),
+                                    v(p["dtr"]), v(p["dtb"]), v(p["x"]), v(p["B"]), v(p["C"]), v(p["dt"]), None)
+    d = _dims(ssd)
+    for over in (dict(xbc=None), dict(w=FAKE + 4), dict(x=FAKE + 8), dict(dt=FAKE + 2), dict(si=FAKE + 2),
+                 dict(so=FAKE + 1), dict(dtb=None), dict(xbc=FAKE + 1)):
+        assert call(d, **over) == ssd.ERR_INVALID_ARG, over
+    assert call(_dims(ssd, b=70000)) == ssd.ERR_INVALID_ARG
+    assert call(_dims(ssd, b=0), xbc=None, w=None, dtr=None, dtb=None, x=None, B=None, C=None, dt=None) == ssd.OK
