@@ -431,8 +431,8 @@ k_state_passing_bf16(const float *__restrict__ states, const float *__restrict__
 // x row anyway, store D x_t / u_t into the intra-chunk accumulator before the MMA adds
 // W X' onto it; the output warps then only combine the two accumulators and hand each
 // [32 rows][32 channels] tile of y to a TMA store.
-constexpr int K3_THREADS = 544;  // warp 0 TMA, 1 MMA (G, inter), 2-5 W/x scaling, 6-13 output, 14 decay-table
-                                 // loads, 15 MMA (intra, source block 0), 16 MMA (intra, source block 1)
+constexpr int K3_THREADS = 672;  // warp 0 TMA, 1 MMA (G, inter), 2-5 and 17-20 W/x scaling, 6-13 output,
+                                 // 14 decay-table loads, 15 MMA (intra, source block 0), 16 MMA (intra, block 1)
 constexpr int K3_CUMBUF = 4;
 constexpr int K3_MAXSLOTS = 5;
 constexpr float kSteepLog2 = 100.f;
@@ -663,13 +663,14 @@ k_chunk_scan_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
       }
     }
     __syncwarp();
-  } else if (warp < 6) {
-    // ------------------------------------------------------------- W build and x scaling (128 threads)
-    // Thread (q, lane) owns row tl = 32q + lane of W and of the accumulators (TMEM lane tl);
-    // the warp's rows are the 32-token group q of the tile.
-    const int q = warp & 3;
+  } else if (warp < 6 || warp >= 17) {
+    // ------------------------------------------------------------- W build and x scaling (256 threads)
+    // Two warps per TMEM lane quarter q: thread (q, hh, lane) owns row tl = 32q + lane of W
+    // and of the accumulators (TMEM lane tl), and the half hh of the columns: W's 32-column
+    // groups 2hh and 2hh + 1, and x's channels 32hh .. 32hh + 31.
+    const int q = warp & 3, hh = warp >= 17 ? 1 : 0;
     const int tl = q * 32 + lane;
-    const int tid = threadIdx.x - 64;
+    const int tid = hh ? (int)threadIdx.x - 17 * 32 + 128 : (int)threadIdx.x - 64;
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
     const int t = 128 * ti + tl;  // chunk-relative row
     const int r = 128 * ti - 1;   // reference token (tile start)
@@ -678,7 +679,7 @@ k_chunk_scan_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
     tc_fence_after();
     if (ok) {
       for (int jj = 0; jj < nblk; ++jj)
-        for (int grp = 0; grp < 4; ++grp) {
+        for (int grp = 2 * hh; grp < 2 * hh + 2; ++grp) {
           const int col0 = 128 * jj + 32 * grp;  // chunk-relative first source column
           uint32_t pk[16];
           if (jj == ti && grp > q) {  // strictly right of the diagonal
@@ -700,7 +701,7 @@ k_chunk_scan_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
       tmem_st_wait();
     }
     tc_fence_before();
-    named_barrier(1, 128);
+    named_barrier(1, 256);
     if (tid == 0 && ok) mbar_arrive(&ms->w_ready);
     bool prev_steep = false;
     for (int k = 0; k < nh; ++k) {
@@ -720,7 +721,7 @@ k_chunk_scan_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
           const float *dts = td.dt;
           const float c2t = c2[t];
           for (int jj = 0; jj < nblk; ++jj)
-            for (int grp = 0; grp < 4; ++grp) {
+            for (int grp = 2 * hh; grp < 2 * hh + 2; ++grp) {
               const int col0 = 128 * jj + 32 * grp;
               uint32_t pk[16];
               if (jj == ti && grp > q) {
@@ -776,8 +777,8 @@ k_chunk_scan_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
           // the column factor in bf16: one packed multiply per pair of channels
           const float vs = ex2(td.c2ref - td.c2[128 * jj + tl]) * td.dt[128 * jj + tl];
           const uint32_t vv2 = pack_bf16x2(vs, vs);
-#pragma unroll
-          for (int half = 0; half < 2; ++half) {  // channels 32 half .. 32 half + 31
+          {
+            const int half = hh;  // channels 32 half .. 32 half + 31
             uint32_t w[16];
 #pragma unroll
             for (int cc = 0; cc < 4; ++cc) {
@@ -814,7 +815,7 @@ k_chunk_scan_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
       }
       fence_proxy_async_smem();
       tc_fence_before();
-      named_barrier(1, 128);
+      named_barrier(1, 256);
       if (tid == 0 && ok) {
         mbar_arrive(&ms->ops_ready[s]);
         mbar_arrive(&ms->cum_free[cb]);
