@@ -210,6 +210,21 @@ SSD_API ssd_status ssd_prefill_noalloc(const ssd_dims *dims, ssd_dtype dtype, co
                                        const float *A, const void *B, const void *C, const float *D, int chunk,
                                        float *y, float *final_state, ssd_stream_t stream);
 
+/*
+ * Self-test of the bounded device-side waits (the library's own check; the pages describe
+ * no such call).  Every mbarrier wait in the tensor-core prefill kernels gives up after a
+ * time limit, sets the workspace's error word and lets the kernel finish, so a lost
+ * producer surfaces as SSD_ERR_TIMEOUT from ssd_prefill_device_status instead of a hung
+ * GPU.  This call runs that same wait in one small kernel: with `expire` non-zero nothing
+ * ever arrives on the barrier and the wait runs out after `limit_ns` (1 .. 1e8 ns); with
+ * `expire` zero the barrier completes at once.  It clears the error word first; read the
+ * outcome with ssd_prefill_device_status (SSD_ERR_TIMEOUT, resp. SSD_OK).  Asynchronous.
+ * Errors: SSD_ERR_INVALID_ARG for a NULL, misaligned or too small workspace or a limit out
+ * of range; SSD_ERR_CUDA if the launch fails.
+ */
+SSD_API ssd_status ssd_wait_selftest(void *workspace, size_t workspace_bytes, uint64_t limit_ns, int expire,
+                                     ssd_stream_t stream);
+
 /* Size in bytes of the fixed scratch array ssd_prefill_noalloc uses (32 MiB). */
 SSD_API size_t ssd_prefill_noalloc_max_workspace(void);
 

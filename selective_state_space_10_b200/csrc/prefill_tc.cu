@@ -282,9 +282,11 @@ k_chunk_state_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
           for (int q = 0; q < 4; ++q) {
             const float a0 = __uint_as_float(in[q] << 16) * wv;  // exact x * w in fp32
             const float a1 = __uint_as_float(in[q] & 0xffff0000u) * wv;
-            hi[q] = pack_bf16x2(a0, a1);
-            const float h0f = __uint_as_float(hi[q] << 16), h1f = __uint_as_float(hi[q] & 0xffff0000u);
-            rem[q] = pack_bf16x2(a0 - h0f, a1 - h1f);
+            // high part: the top 16 bits (truncation), so a - high is exact in fp32 and is
+            // rounded once, to the bf16 remainder
+            const uint32_t b0 = __float_as_uint(a0) & 0xffff0000u, b1 = __float_as_uint(a1) & 0xffff0000u;
+            hi[q] = __byte_perm(b0, b1, 0x7632);
+            rem[q] = pack_bf16x2(a0 - __uint_as_float(b0), a1 - __uint_as_float(b1));
           }
           st_shared_v4(xs + off, hi[0], hi[1], hi[2], hi[3]);
           st_shared_v4(ls + off, rem[0], rem[1], rem[2], rem[3]);

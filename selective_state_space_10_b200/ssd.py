@@ -35,7 +35,7 @@ EXPORTS = ("ssd_status_string", "ssd_version", "ssd_prefill_workspace_size",
            "ssd_prefill_kernel_launches", "ssd_prefill", "ssd_prefill_ex", "ssd_prefill_timed",
            "ssd_prefill_kernel_name", "ssd_prefill_device_status", "ssd_prefill_noalloc",
            "ssd_prefill_noalloc_max_workspace", "ssd_decode_step", "ssd_frontend", "ssd_decode_window_step",
-           "ssd_decode_window_flush")
+           "ssd_decode_window_flush", "ssd_wait_selftest")
 
 
 def _load():
@@ -70,6 +70,8 @@ def _load():
     lib.ssd_prefill_noalloc_max_workspace.restype = sz
     lib.ssd_decode_step.argtypes = [dp, ci, fp, vp, fp, fp, vp, vp, fp, fp, vp]
     lib.ssd_decode_step.restype = ci
+    lib.ssd_wait_selftest.argtypes = [vp, sz, ctypes.c_uint64, ci, vp]
+    lib.ssd_wait_selftest.restype = ci
     lib.ssd_frontend.argtypes = [dp, ci, vp, fp, fp, fp, fp, fp, fp, vp, vp, vp, fp, vp]
     lib.ssd_frontend.restype = ci
     lib.ssd_decode_window_step.argtypes = [dp, ci, ci, ci, fp, vp, fp, vp, vp, fp, fp, vp, vp, fp, fp, vp]
@@ -379,3 +381,13 @@ def frontend(xbc, conv_w, dt_raw, dt_bias, nheads: int, headdim: int, ngroups: i
     if st != OK:
         raise SSDError(st, "ssd_frontend")
     return x, B, C, dt
+
+
+def wait_selftest(workspace, limit_ns: int = 1_000_000, expire: bool = True, stream=None) -> int:
+    """ssd_wait_selftest, then ssd_prefill_device_status: ERR_TIMEOUT when the bounded
+    device wait ran out (expire=True), OK when it completed."""
+    nbytes = workspace.numel() * workspace.element_size()
+    st = lib.ssd_wait_selftest(_ptr(workspace), nbytes, int(limit_ns), 1 if expire else 0, _stream(stream))
+    if st != OK:
+        raise SSDError(st, "ssd_wait_selftest")
+    return prefill_device_status(workspace, stream)

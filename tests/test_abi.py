@@ -217,3 +217,12 @@ def test_frontend_rejects_invalid(ssd):
         assert call(d, **over) == ssd.ERR_INVALID_ARG, over
     assert call(_dims(ssd, b=70000)) == ssd.ERR_INVALID_ARG
     assert call(_dims(ssd, b=0), xbc=None, w=None, dtr=None, dtb=None, x=None, B=None, C=None, dt=None) == ssd.OK
+
+
+def test_wait_selftest_validation_without_a_gpu(ssd):
+    f = ssd.lib.ssd_wait_selftest
+    assert f(None, 256, 1000000, 1, None) == ssd.ERR_INVALID_ARG
+    assert f(ctypes.c_void_p(FAKE + 4), 256, 1000000, 1, None) == ssd.ERR_INVALID_ARG
+    assert f(ctypes.c_void_p(FAKE), 2, 1000000, 1, None) == ssd.ERR_INVALID_ARG
+    assert f(ctypes.c_void_p(FAKE), 256, 0, 1, None) == ssd.ERR_INVALID_ARG
+    assert f(ctypes.c_void_p(FAKE), 256, 10 ** 9, 1, None) == ssd.ERR_INVALID_ARG

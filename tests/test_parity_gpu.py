@@ -339,3 +339,19 @@ def test_windowed_decode_matches_the_recurrence(ssd, dtype, shape, W):
     for k in range(K):  # per-step bound, as for the decode workloads
         assert_close(y_w[:, k], y_ref[:, L0 + k], tol, f"windowed y at step {k}")
     assert_close(state.cpu().numpy(), st_ref, tol, "state after the windows")
+
+
+# ----------------------------------------------------------------- failure detection
+
+def test_bounded_device_wait_expires_and_the_context_stays_usable(ssd):
+    """A wait that nothing satisfies gives up after its limit and reports SSD_ERR_TIMEOUT
+    through the workspace's error word (no trap, no hang); the same wait satisfied reports
+    OK; a prefill on the same context afterwards still matches the oracle."""
+    import time
+    ws = torch.empty(256, dtype=torch.uint8, device="cuda")
+    t0 = time.perf_counter()
+    assert ssd.wait_selftest(ws, limit_ns=2_000_000, expire=True) == ssd.ERR_TIMEOUT
+    assert time.perf_counter() - t0 < 5.0
+    assert ssd.wait_selftest(ws, limit_ns=2_000_000, expire=False) == ssd.OK
+    si = inputs.sequence(1, 300, 2, 64, 128, 1, "bf16", seed=8)
+    check_prefill(ssd, si, 256, "prefill after an expired wait")
