@@ -477,12 +477,17 @@ static_assert(K3Smem::misc + sizeof(K3Misc) <= K3Smem::ring, "K3Misc overlaps th
 constexpr size_t kK3SmemBytes = 1024 + K3Smem::end;
 
 // One head's decay data for one row tile, read from its table row in shared memory: the
-// reference token's c2 (0 before the chunk) and whether the tile's decay range is too
-// steep for the row/column factorisation.  Every role derives these identically.
+// reference token's c2 (0 before the chunk), and how the tile is factorised:
+//   plain -- the tile's decay range is below 2^100: one reference token for all of it;
+//   split -- the range is wider but each half of the tile's rows (64 tokens) spans less
+//            than 2^100: sources and rows from chunk-relative m = 128*ti + 64 on use the
+//            second reference m - 1 (c2ref2) and accumulate apart from the rest;
+//   steep -- neither: the head gets its own W with the decay folded in per element.
+// Every role derives these identically.
 struct TileDecay {
   const float *c2, *dt;
-  float c2ref, dcoef;
-  bool steep;
+  float c2ref, c2ref2, dcoef;
+  bool split, steep;
 };
 __device__ __forceinline__ TileDecay tile_decay(const float *row, int Q, int ti, int nblk, int valid) {
   TileDecay t;
@@ -491,7 +496,11 @@ __device__ __forceinline__ TileDecay tile_decay(const float *row, int Q, int ti,
   t.dcoef = row[0];
   t.c2ref = ti > 0 ? t.c2[128 * ti - 1] : 0.f;
   const int last = min(valid, 128 * nblk) - 1;
-  t.steep = !(fabsf(t.c2ref - t.c2[last]) < kSteepLog2);  // also catches NaN
+  const int m = 128 * ti + 64;
+  t.c2ref2 = t.c2[m - 1];
+  const bool wide = !(fabsf(t.c2ref - t.c2[last]) < kSteepLog2);  // also catches NaN
+  t.split = wide && m <= last && fabsf(t.c2ref - t.c2ref2) < kSteepLog2 && fabsf(t.c2ref2 - t.c2[last]) < kSteepLog2;
+  t.steep = wide && !t.split;
   return t;
 }
 
@@ -545,10 +554,10 @@ k_chunk_scan_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
     for (int s = 0; s < K3_MAXSLOTS; ++s) {
       mbar_init(&ms->x_full[s], 1);
       mbar_init(&ms->ops_ready[s], 1);
-      mbar_init(&ms->x_free[s], nblk + 1);  // commits of every MMA issuer
+      mbar_init(&ms->x_free[s], 3);  // commits of the three MMA issuers
     }
     for (int a = 0; a < 2; ++a) {
-      mbar_init(&ms->acc_full[a], nblk + 1);  // commits of every MMA issuer
+      mbar_init(&ms->acc_full[a], 3);  // commits of the three MMA issuers
       mbar_init(&ms->acc_free[a], 1);
     }
     for (int s = 0; s < K3_CUMBUF; ++s) {
@@ -772,12 +781,25 @@ k_chunk_scan_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
       if (ok) {
         const uint32_t xs = smem_u32(base + K3Smem::slot(nblk, s));
         const float c2t = td.c2[t];
-        const float dsc = steep ? dh : dh * ex2(td.c2ref - c2t);  // D / u_t
-        const uint32_t acc_i = tmem + lane_off + k3_buf(a) + 64u;
+        // A split head's rows and sources from m = 128*ti + 64 on take the second reference,
+        // and their D x_t / u_t goes to the second intra accumulator (the first gets 0 for
+        // them, and the second gets 0 for the rows before m).
+        const bool second = td.split && tl >= 64;
+        const float dsc = steep ? dh : dh * ex2((second ? td.c2ref2 : td.c2ref) - c2t);  // D / u_t
+        const uint32_t acc_i = tmem + lane_off + k3_buf(a) + (second ? 128u : 64u);
+        if (td.split && ok) {  // the other intra accumulator starts from 0 in this row
+          uint32_t z[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) z[e] = 0u;
+          const uint32_t acc_z = tmem + lane_off + k3_buf(a) + (second ? 64u : 128u) + 32u * (uint32_t)hh;
+          tmem_st16(acc_z, z);
+          tmem_st16(acc_z + 16u, z);
+        }
         for (int jj = 0; jj < nblk; ++jj) {
           const uint32_t ra = xs + (uint32_t)jj * 16384u + (uint32_t)tl * 128u;
           // the column factor in bf16: one packed multiply per pair of channels
-          const float vs = ex2(td.c2ref - td.c2[128 * jj + tl]) * td.dt[128 * jj + tl];
+          const float vref = (second && jj == ti) ? td.c2ref2 : td.c2ref;
+          const float vs = ex2(vref - td.c2[128 * jj + tl]) * td.dt[128 * jj + tl];
           const uint32_t vv2 = pack_bf16x2(vs, vs);
           {
             const int half = hh;  // channels 32 half .. 32 half + 31
@@ -845,18 +867,25 @@ k_chunk_scan_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
       float et = 0.f, ut = 0.f;
       if (ok) {
         const uint32_t acc = tmem + lane_off + k3_buf(a) + 32u * hf;
+        const TileDecay td = tile_decay(ms->tab[cb], Q, ti, nblk, valid);
+        const float c2t = td.c2[t];
+        et = ex2(c2t);
+        ut = td.steep ? 1.f : ex2(c2t - td.c2ref);
         tmem_ld32(acc + 64u, va);
-        if (nblk > 1) {  // the two source blocks' intra-chunk products share the row factor u_t
+        if (td.split) {  // second accumulator: sources from m on, row factor relative to m - 1
+          tmem_ld32(acc + 128u, vi);
+          const float ut2 = ex2(c2t - td.c2ref2);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 32; ++j) va[j] = fmaf(ut2, vi[j], ut * va[j]);
+          ut = 1.f;
+        } else if (nblk > 1) {  // the two source blocks' intra-chunk products share the row factor u_t
           tmem_ld32(acc + 128u, vi);
           tmem_ld_wait();
 #pragma unroll
           for (int j = 0; j < 32; ++j) va[j] += vi[j];
         }
         tmem_ld32(acc, vi);
-        const TileDecay td = tile_decay(ms->tab[cb], Q, ti, nblk, valid);
-        const float c2t = td.c2[t];
-        et = ex2(c2t);
-        ut = td.steep ? 1.f : ex2(c2t - td.c2ref);
         tmem_ld_wait();
       }
       // the accumulators and decay tables are read: release them before writing y
@@ -892,23 +921,36 @@ k_chunk_scan_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
     // Warp 15 forms W_{., 0} X'_0 onto D x / u (stored by the scaling warps), warp 16 the
     // second row tile's W_{., 1} X'_1 into its own accumulator.  ops_ready implies x_full,
     // acc_free and W_base: the scaling warps waited for all three.
-    const int jj = warp - 15;  // source block
-    if (lane == 0 && jj < nblk) {
+    // A split head's K steps are divided at its second reference m = 128*ti + 64 instead:
+    // warp 15 takes every source before m (into the first accumulator), warp 16 the
+    // sources from m on (into the second).  Both warps commit for every head.
+    const int iss = warp - 15;
+    if (lane == 0) {
       const uint32_t id_intra = idesc_bf16_f32(128, TP, false, true);
       for (int k = 0; k < nh; ++k) {
         const int s = k % NS, u = k / NS, a = k & 1, cb = k % K3_CUMBUF;
         if (!mbar_wait(&ms->ops_ready[s], u & 1, abort_flag, err)) break;
         if (!mbar_wait(&ms->tab_full[cb], (k / K3_CUMBUF) & 1, abort_flag, err)) break;  // complete already
         tc_fence_after();
-        const uint32_t acc = tmem + k3_buf(a) + 64u * (uint32_t)(1 + jj);
+        const uint32_t acc = tmem + k3_buf(a) + 64u * (uint32_t)(1 + iss);
         const uint32_t so = smem_u32(base + K3Smem::slot(nblk, s));
         // A from TMEM (W_base, or a steep head's own W in the other buffer), K = source tokens
-        const bool steep = tile_decay(ms->tab[cb], Q, ti, nblk, valid).steep;
-        const uint32_t wa = tmem + (steep ? k3_buf(a ^ 1) : K3_TM_WB) + (uint32_t)(64 * jj);
-        for (int ks = 0; ks < 8; ++ks) {
-          const uint64_t bd = smem_desc_sw128(so + jj * 16384u + ks * 2048u, 16384u, 1024u);
-          // block 0 adds onto D x / u; block 1 starts its own accumulator
-          mma_bf16_ts(acc, wa + (uint32_t)(8 * ks), bd, id_intra, (jj == 0 || ks > 0) ? 1u : 0u);
+        const TileDecay td = tile_decay(ms->tab[cb], Q, ti, nblk, valid);
+        const uint32_t wbase = tmem + (td.steep ? k3_buf(a ^ 1) : K3_TM_WB);
+        // the K steps (16 source tokens each, chunk-relative step index 8*block + ks) of this issuer
+        int ks0, ks1;
+        if (td.split) {
+          ks0 = iss == 0 ? 0 : 8 * ti + 4;
+          ks1 = iss == 0 ? 8 * ti + 4 : 8 * nblk;
+        } else {
+          ks0 = 8 * iss;
+          ks1 = iss < nblk ? 8 * iss + 8 : ks0;  // the first row tile has one source block
+        }
+        for (int kk = ks0; kk < ks1; ++kk) {
+          const uint64_t bd = smem_desc_sw128(so + (uint32_t)(kk >> 3) * 16384u + (uint32_t)(kk & 7) * 2048u, 16384u, 1024u);
+          // the first accumulator (and a split head's second) adds onto D x / u; a plain
+          // head's block-1 accumulator starts from its first step
+          mma_bf16_ts(acc, wbase + (uint32_t)(8 * kk), bd, id_intra, (iss == 0 || td.split || kk > ks0) ? 1u : 0u);
         }
         mma_commit(&ms->acc_full[a]);
         mma_commit(&ms->x_free[s]);

@@ -240,6 +240,27 @@ def _random_state(si, seed):
     return np.random.default_rng(seed).standard_normal((b, H, P, N)) * 0.1
 
 
+@pytest.mark.parametrize("L", [500, 400])
+def test_wide_decay_ranges_take_every_factorisation(ssd, L):
+    """The tensor-core chunk scan factorises a tile's decays three ways: one reference token
+    when the tile's decay spans less than 2^100, two (one per 64-row half) when it spans
+    more but each half less, and the decay folded into W per element otherwise.  Heads
+    built to land in each (log2 ranges per 128 tokens of about 50; 150 and 190 with even
+    halves; 260; and 138 packed into one half, either half) against the recurrence; with
+    L = 500 the last tile is ragged past its split point, with L = 400 before it."""
+    H = 6
+    si = inputs.sequence(1, L, H, 64, 128, 1, "bf16", seed=77)
+    log2e = 1.0 / np.log(2.0)
+    dt = np.full((1, L, H), 0.1, dtype=np.float32)
+    tok = np.arange(L) % 128
+    dt[0, :, 4] = np.where(tok < 64, 0.15, 0.01)
+    dt[0, :, 5] = np.where(tok < 64, 0.01, 0.15)
+    A = -np.array([50.0, 150.0, 190.0, 260.0, 0.0, 0.0]) / (128 * 0.1 * log2e)
+    A[4] = A[5] = -10.0
+    si = replace(si, dt=dt, A=A.astype(np.float32))
+    check_prefill(ssd, si, 256, f"wide decay ranges, L={L}")
+
+
 @pytest.mark.parametrize("dtype,shape", [
     ("bf16", dict(b=2, L=600, H=4, P=64, N=128, G=1, Q=256)),   # tensor-core path, ragged tail
     ("bf16", dict(b=1, L=300, H=4, P=64, N=128, G=2, Q=128)),   # tensor-core path, two groups
