@@ -361,17 +361,28 @@ k_chunk_state_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
 
 // ============================================================================ K2
 // grid (b * H, ceil(P*N/4 / 256)), block 256: one float4 of the state per thread.  The
-// chunk states of 8 chunks are loaded before the sequential update so that their
-// latencies overlap; the state entering chunk c is stored in bf16, the final state in fp32.
-// The recurrence starts from `init` (zero if NULL); with `cstates` non-NULL the state
-// after every chunk is also written there in fp32.  `init` may be final_state: each
-// thread reads its element before it writes it.
-constexpr int K2_BATCH = 8;
+// update is sequential over chunks, so the time goes in waiting for the chunk states: a
+// thread fetches K2_ROUND chunks at once, half into registers and half into shared memory
+// by cp.async (which holds no register), so that a CTA has a whole round in flight after
+// one issue pass and few CTAs per SM cover the layer.  The state entering chunk c is
+// stored in bf16, the final state in fp32.  The recurrence starts from `init` (zero if
+// NULL); with `cstates` non-NULL the state after every chunk is also written there in
+// fp32.  `init` may be final_state: each thread reads its element before it writes it.
+constexpr int K2_THREADS = 256;
+constexpr int K2_REG = 8;              // chunks of a round held in registers
+constexpr int K2_STAGED = 8;           // chunks of a round staged in shared memory
+constexpr int K2_ROUND = K2_REG + K2_STAGED;
+constexpr size_t kK2SmemBytes = (size_t)K2_STAGED * K2_THREADS * sizeof(float4);
 
-__global__ void __launch_bounds__(256)
+__device__ __forceinline__ void cp_async16(void *dst, const void *src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+
+__global__ void __launch_bounds__(K2_THREADS, 4)
 k_state_passing_bf16(const float *__restrict__ states, const float *__restrict__ cdecay,
                      __nv_bfloat16 *__restrict__ hprev, const float *init, float *final_state,
                      float *__restrict__ cstates, Dims d, int nc) {
+  extern __shared__ float4 k2_stage[];  // [K2_STAGED][K2_THREADS]
   const int PN4 = d.P * d.N / 4;
   const int e4 = blockIdx.y * blockDim.x + threadIdx.x;
   sm100::grid_dep_launch();  // the chunk scan may start its own set-up meanwhile
@@ -386,25 +397,33 @@ k_state_passing_bf16(const float *__restrict__ states, const float *__restrict__
   const size_t own4 = ((size_t)bi * d.H + h) * PN4 + e4;  // this element in a [b][H][P][N] state
   float4 hs = init ? reinterpret_cast<const float4 *>(init)[own4] : make_float4(0.f, 0.f, 0.f, 0.f);
   float4 *cs = cstates ? reinterpret_cast<float4 *>(cstates) + off0 : nullptr;
-  for (int c0 = 0; c0 < nc; c0 += K2_BATCH) {
-    float4 sv[K2_BATCH];
-    float dc[K2_BATCH];
+  float4 *stage = k2_stage + threadIdx.x;
+  auto step = [&](int c, const float4 &sv) {
+    const float dc = __ldg(dec + c);
+    hp[(size_t)c * cstride] = make_uint2(sm100::pack_bf16x2(hs.x, hs.y), sm100::pack_bf16x2(hs.z, hs.w));
+    hs.x = fmaf(dc, hs.x, sv.x);
+    hs.y = fmaf(dc, hs.y, sv.y);
+    hs.z = fmaf(dc, hs.z, sv.z);
+    hs.w = fmaf(dc, hs.w, sv.w);
+    if (cs) cs[(size_t)c * cstride] = hs;  // state after chunk c
+  };
+  for (int c0 = 0; c0 < nc; c0 += K2_ROUND) {
+    // issue the whole round: chunks c0 .. c0+7 into registers, c0+8 .. c0+15 into shared memory
 #pragma unroll
-    for (int j = 0; j < K2_BATCH; ++j)
-      if (c0 + j < nc) {
-        sv[j] = __ldcs(sp + (size_t)(c0 + j) * cstride);
-        dc[j] = dec[c0 + j];
-      }
+    for (int j = 0; j < K2_STAGED; ++j)
+      if (c0 + K2_REG + j < nc) cp_async16(stage + j * K2_THREADS, sp + (size_t)(c0 + K2_REG + j) * cstride);
+    asm volatile("cp.async.commit_group;" ::: "memory");
+    float4 sv[K2_REG];
 #pragma unroll
-    for (int j = 0; j < K2_BATCH; ++j)
-      if (c0 + j < nc) {
-        hp[(size_t)(c0 + j) * cstride] = make_uint2(sm100::pack_bf16x2(hs.x, hs.y), sm100::pack_bf16x2(hs.z, hs.w));
-        hs.x = fmaf(dc[j], hs.x, sv[j].x);
-        hs.y = fmaf(dc[j], hs.y, sv[j].y);
-        hs.z = fmaf(dc[j], hs.z, sv[j].z);
-        hs.w = fmaf(dc[j], hs.w, sv[j].w);
-        if (cs) cs[(size_t)(c0 + j) * cstride] = hs;  // state after chunk c0 + j
-      }
+    for (int j = 0; j < K2_REG; ++j)
+      if (c0 + j < nc) sv[j] = __ldcs(sp + (size_t)(c0 + j) * cstride);
+#pragma unroll
+    for (int j = 0; j < K2_REG; ++j)
+      if (c0 + j < nc) step(c0 + j, sv[j]);
+    asm volatile("cp.async.wait_group 0;" ::: "memory");  // this thread's own copies
+#pragma unroll
+    for (int j = 0; j < K2_STAGED; ++j)
+      if (c0 + K2_REG + j < nc) step(c0 + K2_REG + j, stage[j * K2_THREADS]);
   }
   reinterpret_cast<float4 *>(final_state)[own4] = hs;
 }
@@ -1175,8 +1194,8 @@ cudaError_t launch_tc_prefill(const __nv_bfloat16 *x, const float *dt, const flo
   // K2
   {
     const int per_head = d.P * d.N / 4;
-    e = launch_after(dim3(d.b * d.H, (per_head + 255) / 256), 256, 0, st, pdl, k_state_passing_bf16, states, cdecay,
-                     hprev, init, final_state, cstates, d, nc);
+    e = launch_after(dim3(d.b * d.H, (per_head + K2_THREADS - 1) / K2_THREADS), K2_THREADS, kK2SmemBytes, st, pdl,
+                     k_state_passing_bf16, states, cdecay, hprev, init, final_state, cstates, d, nc);
     if (e != cudaSuccess) return e;
   }
   if ((e = mark(2)) != cudaSuccess) return e;
