@@ -22,7 +22,8 @@
 
 namespace ssd {
 
-constexpr int kFeTokens = 8;  // tokens per thread
+// tokens per thread: the staged tile of 3 + tokens rows x 256 V channels stays within 48 KB
+template <typename T> constexpr int fe_tokens() { return sizeof(T) == 2 ? 16 : 8; }
 
 // cp.async of 4, 8 or 16 bytes global -> shared (both addresses aligned to the size)
 template <int BYTES>
@@ -38,7 +39,8 @@ template <typename T> __device__ __forceinline__ T from_f32(float v);
 template <> __device__ __forceinline__ float from_f32<float>(float v) { return v; }
 template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float v) { return __float2bfloat16_rn(v); }
 
-__device__ __forceinline__ float silu_f(float v) { return v / (1.f + __expf(-v)); }
+// v * sigmoid(v) with the fast reciprocal (about 1 ulp; 0 once exp(-v) overflows)
+__device__ __forceinline__ float silu_f(float v) { return v * __fdividef(1.f, 1.f + __expf(-v)); }
 __device__ __forceinline__ float softplus_f(float z) { return z > 20.f ? z : log1pf(__expf(z)); }
 __device__ __forceinline__ void store_out(float *p, float v) { *p = v; }
 __device__ __forceinline__ void store_out(__nv_bfloat16 *p, float v) { *p = __float2bfloat16_rn(v); }
@@ -78,16 +80,17 @@ template <> struct Vec<__nv_bfloat16, 4> {
   }
 };
 
-// One thread per (V channels, kFeTokens-token run): grid (token runs, channel tiles of
+// One thread per (V channels, fe_tokens<T>()-token run): grid (token runs, channel tiles of
 // 256 * V, batch rows).  V = 4 needs H * P to be a multiple of 4 (then no group of four
 // straddles the x | B | C boundaries, and every vector access is aligned).
 template <typename T, int V>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(256, 4)
 k_frontend(const T *__restrict__ xbc, const float *__restrict__ w, const float *__restrict__ bias,
            const float *__restrict__ state_in, const float *dt_raw, const float *__restrict__ dt_bias,
            T *__restrict__ x, T *__restrict__ B, T *__restrict__ C, float *dt, Dims d) {
   const int HP = d.H * d.P, GN = d.G * d.N, CH = HP + 2 * GN;
   const int c = (blockIdx.y * blockDim.x + threadIdx.x) * V;
+  constexpr int kFeTokens = fe_tokens<T>();
   const int t0 = blockIdx.x * kFeTokens, bi = blockIdx.z;
   const int t1 = min(t0 + kFeTokens, d.L);
   if (blockIdx.y == 0) {  // dt for this run of tokens (all loads issued before any use)
@@ -196,7 +199,7 @@ cudaError_t launch_frontend(const T *xbc, const float *w, const float *bias, con
   const int CH = d.H * d.P + 2 * d.G * d.N;
   // token runs on x (up to 2^31 - 1), channel tiles on y and batch rows on z (the host
   // checks both stay within 65535)
-  const unsigned runs = (unsigned)((d.L + kFeTokens - 1) / kFeTokens);
+  const unsigned runs = (unsigned)((d.L + fe_tokens<T>() - 1) / fe_tokens<T>());
   if ((d.H * d.P) % 4 == 0)
     k_frontend<T, 4><<<dim3(runs, (unsigned)((CH / 4 + 255) / 256), (unsigned)d.b), 256, 0, st>>>(
         xbc, w, bias, state_in, dt_raw, dt_bias, x, B, C, dt, d);
