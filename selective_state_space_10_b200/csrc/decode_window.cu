@@ -76,6 +76,22 @@ k_decode_window_step(const float *__restrict__ state, T *__restrict__ win_x, flo
   const T *Cg = C + ((size_t)bi * d.G + g) * N;
   const float4 *st = reinterpret_cast<const float4 *>(state) + (size_t)bh * d.P * NV;
 
+  // The first pass of the state (the whole of it for P <= 8 * ROWS) and C are loaded
+  // before the window bookkeeping, so that the step's HBM traffic is in flight while the
+  // window terms are formed.
+  float4 cv[VPL];
+#pragma unroll
+  for (int v = 0; v < VPL; ++v) cv[v] = load4(Cg + (size_t)(v * LPR + l) * 4);
+  float4 hv[UNR][VPL];
+#pragma unroll
+  for (int u = 0; u < UNR; ++u) {
+    const int row = u * ROWS + warp * RPW + sub;
+    if (row < d.P) {
+#pragma unroll
+      for (int v = 0; v < VPL; ++v) hv[u][v] = __ldcs(st + (size_t)row * NV + v * LPR + l);
+    }
+  }
+
   // Every global load of the window bookkeeping is issued here, before any of it is
   // used: the window's dt (warp 0), the B_s rows of the C . B_s dots (warp w: tokens w
   // and w + 8) and the window's x values (kStage per thread, more only when P > 128).
@@ -145,17 +161,15 @@ k_decode_window_step(const float *__restrict__ state, T *__restrict__ win_x, flo
 
   float *yh = y + (size_t)bh * d.P;
   const float Dh = D[h], tot = dec[kWinMax];
-  float4 cv[VPL];
-#pragma unroll
-  for (int v = 0; v < VPL; ++v) cv[v] = load4(Cg + (size_t)(v * LPR + l) * 4);
   for (int r0 = 0; r0 < d.P; r0 += ROWS * UNR) {
-    float4 hv[UNR][VPL];
+    if (r0 > 0) {  // later passes (P > 8 * ROWS)
 #pragma unroll
-    for (int u = 0; u < UNR; ++u) {
-      const int row = r0 + u * ROWS + warp * RPW + sub;
-      if (row < d.P) {
+      for (int u = 0; u < UNR; ++u) {
+        const int row = r0 + u * ROWS + warp * RPW + sub;
+        if (row < d.P) {
 #pragma unroll
-        for (int v = 0; v < VPL; ++v) hv[u][v] = __ldcs(st + (size_t)row * NV + v * LPR + l);
+          for (int v = 0; v < VPL; ++v) hv[u][v] = __ldcs(st + (size_t)row * NV + v * LPR + l);
+        }
       }
     }
 #pragma unroll
