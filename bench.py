@@ -24,6 +24,7 @@ only), on a bounded sample of the same workload per step.
 """
 import argparse
 import hashlib
+import re
 import json
 import os
 import statistics
@@ -172,10 +173,15 @@ class ClockSampler:
 
 
 def source_digest(files):
+    """Digest of the code in `files` with comments and whitespace removed, so that a change
+    to a comment does not void counters taken from unchanged kernels."""
     h = hashlib.sha256()
     for f in files:
-        with open(os.path.join(ROOT, f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, f), encoding="utf-8") as fh:
+            text = fh.read()
+        text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", " ", text)
+        h.update(" ".join(text.split()).encode())
     return h.hexdigest()[:16]
 
 

@@ -13,7 +13,8 @@
 //                        kept in shared memory and written out head-major as one table row
 //                        per (batch, head, chunk) for the chunk-scan kernel, plus the
 //                        chunk's total decay 2^c2_end for state passing.  Then, per head
-//                        (ring of 3 x slots), eight warps scale x's rows by the decay weight in fp32 and
+//                        (ring of 3 x slots), eight warps scale x's rows by the decay
+//                        weight in fp32 and
 //                        split the product into a bf16 high part and a bf16 remainder,
 //                        stored side by side; one thread issues tcgen05.mma with both as
 //                        the two 64-wide halves of N = 128 (M = 128 d_state rows, K = Q
@@ -28,10 +29,10 @@
 //                        heads), decay data from K1's table.  G = C_tile B_chunk^T is
 //                        computed once into TMEM and, masked, converted once to a
 //                        head-independent bf16 W (see the decay factorisation at K3
-//                        below); per head, 4 warps scale the
-//                        rows of its x tile by the column decay factors, tcgen05.mma forms
-//                        ACC_inter = C_tile h_prev^T and ACC_intra = W X' (double-buffered
-//                        in TMEM across heads), and 8 warps write
+//                        below); per head, 8 warps scale the rows of its x tile by the
+//                        column decay factors, three threads issue tcgen05.mma for
+//                        ACC_inter = C_tile h_prev^T and the intra-chunk products W X'
+//                        (double-buffered in TMEM across heads), and 8 warps write
 //                        y_t = exp(cum_t) ACC_inter + u_t ACC_intra + D x_t (fp32).
 //
 // Numerics: every decay exp(cum_t - cum_s), s <= t, is formed so that no intermediate
