@@ -440,10 +440,21 @@ def prefill_leg(args, dev, rank, world, peaks, sampler):
     return res
 
 
+def decode_workload(args):
+    """The batched decode workload, or the same shapes at another batch (--decode-batch:
+    a smaller state for profiling captures that must fit a few GB)."""
+    from dataclasses import replace
+    from selective_state_space_10_b200 import inputs
+    w = inputs.BY_NAME[DECODE_WORKLOAD]
+    if args.decode_batch and args.decode_batch != w.batch:
+        w = replace(w, batch=args.decode_batch, name=f"{w.name}@batch{args.decode_batch}")
+    return w
+
+
 def decode_leg(args, dev, rank, world, peaks, sampler):
     import torch
     from selective_state_space_10_b200 import inputs, ssd
-    w = inputs.BY_NAME[DECODE_WORKLOAD]
+    w = decode_workload(args)
     seed = rank_seed(w.seed, rank)
     nsteps = args.decode_steps
     state = torch.from_numpy(inputs.decode_initial_state(w, seed=seed)).to(dev)
@@ -779,7 +790,7 @@ def run_ours(args):
         out["cpu_baseline"] = {"value": rate, "unit": "tokens/s", "cores": threads, "kind": "oracle",
                                "sample": desc, "seconds": secs}
         if dec:
-            wd = inputs.BY_NAME[DECODE_WORKLOAD]
+            wd = decode_workload(args)
             drate, ddesc, dthreads, dsecs = oracle_decode_rate(wd, wd.seed)
             out["decode"]["cpu_baseline"] = {"value": drate, "unit": "steps/s", "cores": dthreads,
                                              "kind": "oracle", "sample": ddesc, "seconds": dsecs}
@@ -835,6 +846,8 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=PREFILL_WORKLOAD)
     ap.add_argument("--decode-steps", type=int, default=1024)
+    ap.add_argument("--decode-batch", type=int, default=None,
+                    help="decode batch (default: the workload's 256); for small profiling captures")
     ap.add_argument("--skip-decode", action="store_true")
     ap.add_argument("--skip-cpu-baseline", action="store_true")
     ap.add_argument("--skip-recompute", action="store_true",
