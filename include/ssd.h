@@ -229,6 +229,30 @@ SSD_API ssd_status ssd_wait_selftest(void *workspace, size_t workspace_bytes, ui
 SSD_API size_t ssd_prefill_noalloc_max_workspace(void);
 
 /*
+ * The prefill end to end, with HOST arrays: copies x, dt, A, B, C and D to the device,
+ * runs ssd_prefill there, and copies y and final_state back, all enqueued on `stream`
+ * in that order (one cudaMemcpyAsync per array).  Arguments, layouts and results are
+ * those of ssd_prefill, except that every array pointer is a host pointer; host arrays
+ * need no particular alignment.  In page-locked host memory the copies run
+ * asynchronously and the call returns once they are enqueued; the host outputs are
+ * complete when the stream has passed the call.  Pageable host memory also works, with
+ * the copies then synchronous with the host.
+ *
+ * device_buffer: caller-owned device memory of at least
+ * ssd_prefill_host_buffer_size(dims, dtype, chunk) bytes, 16-byte aligned: it holds the
+ * device copies of the inputs and outputs and the prefill's workspace.  Calls that share
+ * it must be ordered.
+ *
+ * Errors: as ssd_prefill; SSD_ERR_WORKSPACE if device_buffer is NULL, misaligned or
+ * short.  Nothing is enqueued on an error found before the first copy.
+ */
+SSD_API size_t ssd_prefill_host_buffer_size(const ssd_dims *dims, ssd_dtype dtype, int chunk);
+SSD_API ssd_status ssd_prefill_host(const ssd_dims *dims, ssd_dtype dtype, const void *x, const float *dt,
+                                    const float *A, const void *B, const void *C, const float *D, int chunk,
+                                    float *y, float *final_state, void *device_buffer,
+                                    size_t device_buffer_bytes, ssd_stream_t stream);
+
+/*
  * One cached decode step (O(1) in the sequence length: "Compiler-First State Space
  * Duality ..." abstract; the recurrent mode of "Mamba and Selective State Space Models"
  * section 3).  Reads state = h_{t-1}, overwrites it in place with h_t, writes y_t.

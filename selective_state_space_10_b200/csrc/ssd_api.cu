@@ -238,6 +238,90 @@ ssd_status ssd_prefill_timed(const ssd_dims *dims, ssd_dtype dtype, const void *
                       workspace_bytes, stream, events, num_events, true);
 }
 
+namespace {
+// Offsets in ssd_prefill_host's device buffer: the input copies, the outputs, then the
+// prefill workspace, each 256-byte aligned.
+struct HostPlan {
+  int64_t nx, ndt, nbc, ny, nst;  // element counts
+  size_t esz;
+  size_t x, dt, A, B, C, D, y, fs, ws, ws_bytes, bytes;
+};
+bool plan_host(const ssd_dims *dims, ssd_dtype dtype, int chunk, HostPlan *hp) {
+  Dims d;
+  if (check_dims(dims, dtype, true, &d) != SSD_OK || !is_pow2(chunk) || chunk > 256) return false;
+  const int64_t ntok = (int64_t)d.b * d.L;
+  hp->esz = dtype == SSD_F32 ? 4 : 2;
+  hp->nx = ntok * d.H * d.P;
+  hp->ndt = ntok * d.H;
+  hp->nbc = ntok * d.G * d.N;
+  hp->ny = hp->nx;
+  hp->nst = (int64_t)d.b * d.H * d.P * d.N;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off += align_up(bytes);
+    return at;
+  };
+  hp->x = take((size_t)hp->nx * hp->esz);
+  hp->dt = take((size_t)hp->ndt * 4);
+  hp->A = take((size_t)d.H * 4);
+  hp->B = take((size_t)hp->nbc * hp->esz);
+  hp->C = take((size_t)hp->nbc * hp->esz);
+  hp->D = take((size_t)d.H * 4);
+  hp->y = take((size_t)hp->ny * 4);
+  hp->fs = take((size_t)hp->nst * 4);
+  hp->ws_bytes = plan_prefill(d, dtype, chunk).bytes;
+  hp->ws = take(hp->ws_bytes);
+  hp->bytes = off;
+  return true;
+}
+}  // namespace
+
+size_t ssd_prefill_host_buffer_size(const ssd_dims *dims, ssd_dtype dtype, int chunk) {
+  HostPlan hp;
+  return plan_host(dims, dtype, chunk, &hp) ? hp.bytes : 0;
+}
+
+ssd_status ssd_prefill_host(const ssd_dims *dims, ssd_dtype dtype, const void *x, const float *dt, const float *A,
+                            const void *B, const void *C, const float *D, int chunk, float *y, float *final_state,
+                            void *device_buffer, size_t device_buffer_bytes, ssd_stream_t stream) {
+  Dims d;
+  ssd_status s = check_dims(dims, dtype, true, &d);
+  if (s != SSD_OK) return s;
+  if (!is_pow2(chunk) || chunk > 256) return SSD_ERR_INVALID_ARG;
+  HostPlan hp;
+  if (!plan_host(dims, dtype, chunk, &hp)) return SSD_ERR_INVALID_ARG;
+  // host arrays: non-NULL when non-empty, no alignment needed
+  if ((hp.nx > 0 && (x == nullptr || y == nullptr)) || (hp.ndt > 0 && dt == nullptr) ||
+      (hp.nbc > 0 && (B == nullptr || C == nullptr)) || (hp.nst > 0 && final_state == nullptr) ||
+      (d.b > 0 && (A == nullptr || D == nullptr)))
+    return SSD_ERR_INVALID_ARG;
+  if (d.b == 0) return SSD_OK;  // nothing to compute or copy
+  if (device_buffer == nullptr || !aligned(device_buffer, 16) || device_buffer_bytes < hp.bytes)
+    return SSD_ERR_WORKSPACE;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t *dev = static_cast<uint8_t *>(device_buffer);
+  auto h2d = [&](size_t off, const void *src, size_t bytes) {
+    return bytes == 0 ? cudaSuccess : cudaMemcpyAsync(dev + off, src, bytes, cudaMemcpyHostToDevice, st);
+  };
+  cudaError_t e = h2d(hp.x, x, (size_t)hp.nx * hp.esz);
+  if (e == cudaSuccess) e = h2d(hp.dt, dt, (size_t)hp.ndt * 4);
+  if (e == cudaSuccess) e = h2d(hp.A, A, d.b > 0 ? (size_t)d.H * 4 : 0);
+  if (e == cudaSuccess) e = h2d(hp.B, B, (size_t)hp.nbc * hp.esz);
+  if (e == cudaSuccess) e = h2d(hp.C, C, (size_t)hp.nbc * hp.esz);
+  if (e == cudaSuccess) e = h2d(hp.D, D, d.b > 0 ? (size_t)d.H * 4 : 0);
+  if (e != cudaSuccess) return cuda_status(e);
+  s = ssd_prefill(dims, dtype, dev + hp.x, reinterpret_cast<const float *>(dev + hp.dt),
+                  reinterpret_cast<const float *>(dev + hp.A), dev + hp.B, dev + hp.C,
+                  reinterpret_cast<const float *>(dev + hp.D), chunk, reinterpret_cast<float *>(dev + hp.y),
+                  reinterpret_cast<float *>(dev + hp.fs), dev + hp.ws, hp.ws_bytes, stream);
+  if (s != SSD_OK) return s;
+  if (hp.ny > 0) e = cudaMemcpyAsync(y, dev + hp.y, (size_t)hp.ny * 4, cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess && hp.nst > 0)
+    e = cudaMemcpyAsync(final_state, dev + hp.fs, (size_t)hp.nst * 4, cudaMemcpyDeviceToHost, st);
+  return cuda_status(e);
+}
+
 const char *ssd_prefill_kernel_name(const ssd_dims *dims, ssd_dtype dtype, int chunk, int i) {
   Dims d;
   if (check_dims(dims, dtype, true, &d) != SSD_OK || !is_pow2(chunk) || chunk > 256) return nullptr;

@@ -35,7 +35,7 @@ EXPORTS = ("ssd_status_string", "ssd_version", "ssd_prefill_workspace_size",
            "ssd_prefill_kernel_launches", "ssd_prefill", "ssd_prefill_ex", "ssd_prefill_timed",
            "ssd_prefill_kernel_name", "ssd_prefill_device_status", "ssd_prefill_noalloc",
            "ssd_prefill_noalloc_max_workspace", "ssd_decode_step", "ssd_frontend", "ssd_decode_window_step",
-           "ssd_decode_window_flush", "ssd_wait_selftest")
+           "ssd_decode_window_flush", "ssd_wait_selftest", "ssd_prefill_host_buffer_size", "ssd_prefill_host")
 
 
 def _load():
@@ -68,6 +68,10 @@ def _load():
     lib.ssd_prefill_noalloc.restype = ci
     lib.ssd_prefill_noalloc_max_workspace.argtypes = []
     lib.ssd_prefill_noalloc_max_workspace.restype = sz
+    lib.ssd_prefill_host_buffer_size.argtypes = [dp, ci, ci]
+    lib.ssd_prefill_host_buffer_size.restype = sz
+    lib.ssd_prefill_host.argtypes = [dp, ci, vp, fp, fp, vp, vp, fp, ci, fp, fp, vp, sz, vp]
+    lib.ssd_prefill_host.restype = ci
     lib.ssd_decode_step.argtypes = [dp, ci, fp, vp, fp, fp, vp, vp, fp, fp, vp]
     lib.ssd_decode_step.restype = ci
     lib.ssd_wait_selftest.argtypes = [vp, sz, ctypes.c_uint64, ci, vp]
@@ -209,6 +213,50 @@ def prefill(x, dt, A, B, C, D, chunk: int = 256, y=None, final_state=None, works
     return y, final_state
 
 
+def prefill_host_buffer_size(dims: Dims, dtype: int, chunk: int) -> int:
+    return int(lib.ssd_prefill_host_buffer_size(ctypes.byref(dims), int(dtype), int(chunk)))
+
+
+def prefill_host(x, dt, A, B, C, D, chunk: int = 256, y=None, final_state=None, device_buffer=None,
+                 stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """ssd_prefill_host: the prefill end to end from host tensors (page-locked for
+    asynchronous copies).  The library copies the inputs to `device_buffer` (a CUDA uint8
+    tensor of at least prefill_host_buffer_size() bytes; allocated if None), runs the
+    prefill, and copies y and final_state into host tensors, all on `stream`.  Returns the
+    host (y, final_state); read them after synchronising the stream."""
+    if x.dim() != 4 or B.dim() != 4:
+        raise ValueError("x must be [b,L,H,P] and B, C [b,L,G,N]")
+    if x.dtype not in _DTYPES:
+        raise ValueError(f"unsupported input dtype {x.dtype}")
+    host = torch.device("cpu")
+    b, L, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    for t, name, shape, dtype in ((x, "x", (b, L, H, P), x.dtype), (dt, "dt", (b, L, H), torch.float32),
+                                  (A, "A", (H,), torch.float32), (B, "B", (b, L, G, N), x.dtype),
+                                  (C, "C", (b, L, G, N), x.dtype), (D, "D", (H,), torch.float32)):
+        _check(t, name, shape, dtype, host)
+    pin = x.is_pinned()
+    if y is None:
+        y = torch.empty((b, L, H, P), dtype=torch.float32, pin_memory=pin)
+    if final_state is None:
+        final_state = torch.empty((b, H, P, N), dtype=torch.float32, pin_memory=pin)
+    _check(y, "y", (b, L, H, P), torch.float32, host)
+    _check(final_state, "final_state", (b, H, P, N), torch.float32, host)
+    dims = dims_of_prefill(x, B)
+    dtype = _DTYPES[x.dtype]
+    need = prefill_host_buffer_size(dims, dtype, chunk)
+    if device_buffer is None:
+        device_buffer = torch.empty(max(need, 1), dtype=torch.uint8, device="cuda")
+    if device_buffer.device.type != "cuda":
+        raise ValueError("device_buffer must be a CUDA tensor")
+    st = lib.ssd_prefill_host(ctypes.byref(dims), dtype, _ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
+                              int(chunk), _ptr(y), _ptr(final_state), _ptr(device_buffer),
+                              device_buffer.numel() * device_buffer.element_size(), _stream(stream))
+    if st != OK:
+        raise SSDError(st, "ssd_prefill_host")
+    return y, final_state
+
+
 def prefill_noalloc(x, dt, A, B, C, D, chunk: int = 256, y=None, final_state=None,
                     stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
     """ssd_prefill_noalloc: the same prefill, with no workspace argument.  For callers
@@ -277,22 +325,6 @@ def decode_step(state, x, dt, A, B, C, D, y=None, stream=None) -> torch.Tensor:
     if st != OK:
         raise SSDError(st, "ssd_decode_step")
     return y
-
-
-def prefill_host(x, dt, A, B, C, D, chunk: int = 256, device="cuda", stream=None):
-    """End-to-end prefill from host tensors: copies the inputs to the device, runs
-    ssd_prefill and copies y and the final state back into pinned host tensors.
-    Returns (y_host, final_state_host); the copies are ordered on `stream`."""
-    dev = torch.device(device)
-    s = stream or torch.cuda.current_stream(dev)
-    with torch.cuda.stream(s):
-        d_in = [t.to(dev, non_blocking=True) for t in (x, dt, A, B, C, D)]
-        y, fs = prefill(*d_in, chunk=chunk, stream=s)
-        y_h = torch.empty(y.shape, dtype=y.dtype, pin_memory=True)
-        fs_h = torch.empty(fs.shape, dtype=fs.dtype, pin_memory=True)
-        y_h.copy_(y, non_blocking=True)
-        fs_h.copy_(fs, non_blocking=True)
-    return y_h, fs_h
 
 
 def window_buffers(state: torch.Tensor, window: int, dtype=torch.bfloat16, ngroups: int = 1):

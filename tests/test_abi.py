@@ -226,3 +226,25 @@ def test_wait_selftest_validation_without_a_gpu(ssd):
     assert f(ctypes.c_void_p(FAKE), 2, 1000000, 1, None) == ssd.ERR_INVALID_ARG
     assert f(ctypes.c_void_p(FAKE), 256, 0, 1, None) == ssd.ERR_INVALID_ARG
     assert f(ctypes.c_void_p(FAKE), 256, 10 ** 9, 1, None) == ssd.ERR_INVALID_ARG
+
+
+def test_prefill_host_validation_without_a_gpu(ssd):
+    """ssd_prefill_host checks its arguments and the device buffer before any copy; host
+    arrays need no alignment, the device buffer 16 bytes."""
+    f = ssd.lib.ssd_prefill_host
+    d = _dims(ssd)
+    h = ctypes.c_void_p(FAKE + 2)
+    dev = ctypes.c_void_p(FAKE)
+    need = ssd.prefill_host_buffer_size(d, 1, 256)
+    assert need > ssd.prefill_workspace_size(d, 1, 256)
+    call = lambda dims, x=h, chunk=256, buf=dev, nbytes=need: f(dims, 1, x, h, h, h, h, h, chunk, h, h, buf, nbytes,
+                                                                 None)
+    assert call(None) == ssd.ERR_INVALID_ARG
+    assert call(ctypes.byref(d), chunk=48) == ssd.ERR_INVALID_ARG
+    assert call(ctypes.byref(d), x=None) == ssd.ERR_INVALID_ARG
+    assert call(ctypes.byref(_dims(ssd, N=48))) == ssd.ERR_UNSUPPORTED
+    assert call(ctypes.byref(d), buf=None) == ssd.ERR_WORKSPACE
+    assert call(ctypes.byref(d), nbytes=need - 1) == ssd.ERR_WORKSPACE
+    assert call(ctypes.byref(d), buf=ctypes.c_void_p(FAKE + 8)) == ssd.ERR_WORKSPACE
+    e = _dims(ssd, b=0)
+    assert f(ctypes.byref(e), 1, None, None, None, None, None, None, 256, None, None, None, 0, None) == ssd.OK

@@ -240,6 +240,26 @@ def _random_state(si, seed):
     return np.random.default_rng(seed).standard_normal((b, H, P, N)) * 0.1
 
 
+@pytest.mark.parametrize("dtype,shape", [
+    ("bf16", dict(b=2, L=600, H=4, P=64, N=128, G=1, Q=256)),   # tensor-core path
+    ("f32", dict(b=1, L=200, H=3, P=32, N=64, G=1, Q=64)),      # CUDA-core path
+])
+def test_prefill_host_equals_the_device_call(ssd, dtype, shape):
+    """ssd_prefill_host (host arrays in and out, the copies enqueued by the library) gives
+    exactly the results of ssd_prefill on device copies, from page-locked and from
+    pageable host memory."""
+    s = shape
+    si = inputs.sequence(s["b"], s["L"], s["H"], s["P"], s["N"], s["G"], dtype, seed=404)
+    t = to_device(si)
+    y, fs = ssd.prefill(**t, chunk=s["Q"])
+    torch.cuda.synchronize()
+    for pinned in (True, False):
+        host = {k: (v.cpu().pin_memory() if pinned else v.cpu()) for k, v in t.items()}
+        yh, fsh = ssd.prefill_host(**host, chunk=s["Q"])
+        torch.cuda.synchronize()
+        assert torch.equal(yh, y.cpu()) and torch.equal(fsh, fs.cpu())
+
+
 @pytest.mark.parametrize("L", [500, 400])
 def test_wide_decay_ranges_take_every_factorisation(ssd, L):
     """The tensor-core chunk scan factorises a tile's decays three ways: one reference token
