@@ -18,9 +18,9 @@
 //
 // Both kernels: one CTA of 256 threads per (batch row, head); state rows are covered as
 // in the single-step decode kernel (LPR lanes per row with float4 accesses, all loads of
-// a pass in flight before any arithmetic).  The window's tokens are first staged in
-// shared memory (every thread's loads issued together), already weighted by their decay
-// coefficients.  Window lengths up to 16.
+// a pass in flight before any arithmetic).  The step issues its state loads first and
+// forms the window's terms while they fly; the flush stages the window's tokens in shared
+// memory, already weighted by their decay coefficients.  Window lengths up to 16.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -28,7 +28,6 @@ namespace ssd {
 
 constexpr int kWinMax = 16;
 constexpr int kPMax = 256;
-constexpr int kStage = 8;  // window values each thread loads up front (covers P <= 128)
 
 // The window's decay scan, by the 32 lanes of one warp (lane s holds dt_s, 0 past the
 // window's n tokens): dec[s] = exp(cum_last - cum_s) dt_s for s < n and
@@ -60,9 +59,7 @@ k_decode_window_step(const float *__restrict__ state, T *__restrict__ win_x, flo
   constexpr int UNR = (8 / (RPW * VPL)) > 0 ? 8 / (RPW * VPL) : 1;
   __shared__ float dec[kWinMax + 1];    // exp(cum_pos - cum_s) dt_s; [kWinMax]: exp(cum_pos)
   __shared__ float qs[kWinMax];         // C . B_s
-  extern __shared__ float dyn[];        // (pos + 1) x P floats:
-  float *wsum = dyn;                    //   [P] the window's sum, this token included
-  float *wx = dyn + d.P;                //   [pos][P] coef_s x_s[p] of the window's earlier tokens
+  __shared__ float wsum[kPMax];         // the window's sum, this token included
 
   const int bh = blockIdx.x;
   const int bi = bh / d.H, h = bh - bi * d.H;
@@ -94,7 +91,9 @@ k_decode_window_step(const float *__restrict__ state, T *__restrict__ win_x, flo
 
   // Every global load of the window bookkeeping is issued here, before any of it is
   // used: the window's dt (warp 0), the B_s rows of the C . B_s dots (warp w: tokens w
-  // and w + 8) and the window's x values (kStage per thread, more only when P > 128).
+  // and w + 8) and the window's x values.  For the window sum, four threads share a channel
+  // (thread 4p' + j of a block of 64 channels holds x_s for s = j, j + 4, j + 8, j + 12)
+  // and add their partial sums with two shuffles, so no thread walks the whole window.
   float dts = 0.f;
   if (warp == 0 && lane < n) dts = lane < pos ? win_dt[(wtok + lane) * d.H + h] : dtv;
   float q[2] = {0.f, 0.f};
@@ -110,17 +109,14 @@ k_decode_window_step(const float *__restrict__ state, T *__restrict__ win_x, flo
       }
     }
   }
-  const int nstage = pos * d.P;
   const T *wxh = win_x + (wtok * d.H + h) * (size_t)d.P;  // slot s of this head at s * H * P
-  float xr[kStage];
+  const T *xh = x + (size_t)bh * d.P;
+  const int pj = threadIdx.x >> 2, jw = threadIdx.x & 3;   // channel within a block of 64, window phase
+  float xw[kWinMax / 4];
 #pragma unroll
-  for (int j = 0; j < kStage; ++j) {
-    const int i = threadIdx.x + 256 * j;
-    xr[j] = 0.f;
-    if (i < nstage) {
-      const int s = i / d.P;
-      xr[j] = to_f32(wxh[(size_t)s * d.H * d.P + (i - s * d.P)]);
-    }
+  for (int i = 0; i < kWinMax / 4; ++i) {  // the first block of channels, loaded up front
+    const int s = jw + 4 * i;
+    xw[i] = (pj < d.P && s < pos) ? to_f32(wxh[(size_t)s * d.H * d.P + pj]) : 0.f;
   }
   if (warp == 0) window_decays(n, Ah, dts, dec);  // dec[s] = exp(cum_pos - cum_s) dt_s, dec[kWinMax] = exp(cum_pos)
 #pragma unroll
@@ -129,25 +125,25 @@ k_decode_window_step(const float *__restrict__ state, T *__restrict__ win_x, flo
     if (lane == 0 && warp + 8 * j < n) qs[warp + 8 * j] = qq;
   }
   __syncthreads();
-  // coef_s = dec[s] * (C . B_s); the earlier tokens' weighted x into shared memory
+  // wsum[p] = sum_{s <= pos} dec_s (C . B_s) x_s[p]
+  for (int pb = 0; pb < d.P; pb += 64) {
+    const int p = pb + pj;
+    if (pb > 0) {  // later blocks (P > 64)
 #pragma unroll
-  for (int j = 0; j < kStage; ++j) {
-    const int i = threadIdx.x + 256 * j;
-    if (i < nstage) {
-      const int s = i / d.P;
-      wx[i] = dec[s] * qs[s] * xr[j];  // wx[s][p] at s * P + p = i
+      for (int i = 0; i < kWinMax / 4; ++i) {
+        const int s = jw + 4 * i;
+        xw[i] = (p < d.P && s < pos) ? to_f32(wxh[(size_t)s * d.H * d.P + p]) : 0.f;
+      }
     }
-  }
-  for (int i = threadIdx.x + 256 * kStage; i < nstage; i += blockDim.x) {  // P > 128 only
-    const int s = i / d.P;
-    wx[i] = dec[s] * qs[s] * to_f32(wxh[(size_t)s * d.H * d.P + (i - s * d.P)]);
-  }
-  const T *xh = x + (size_t)bh * d.P;
-  __syncthreads();
-  for (int p = threadIdx.x; p < d.P; p += blockDim.x) {
-    float w = dec[pos] * qs[pos] * to_f32(xh[p]);
-    for (int s = 0; s < pos; ++s) w += wx[s * d.P + p];
-    wsum[p] = w;
+    float part = 0.f;
+#pragma unroll
+    for (int i = 0; i < kWinMax / 4; ++i) {
+      const int s = jw + 4 * i;
+      if (s < pos) part = fmaf(dec[s] * qs[s], xw[i], part);
+    }
+    part += __shfl_xor_sync(0xffffffffu, part, 1);
+    part += __shfl_xor_sync(0xffffffffu, part, 2);
+    if (jw == 0 && p < d.P) wsum[p] = fmaf(dec[pos] * qs[pos], to_f32(xh[p]), part);
   }
   __syncthreads();
 
@@ -323,9 +319,8 @@ cudaError_t launch_decode_window_step(const float *state, T *win_x, float *win_d
                                       const T *x, const float *dt, const float *A, const T *B, const T *C,
                                       const float *D, float *y, const Dims &d, cudaStream_t st) {
   const dim3 grid((unsigned)((size_t)d.b * d.H));
-  const size_t smem = (size_t)(pos + 1) * d.P * sizeof(float);
 #define SSD_WSTEP(NN)                                                                                              \
-  k_decode_window_step<T, NN><<<grid, 256, smem, st>>>(state, win_x, win_dt, win_B, W, pos, x, dt, A, B, C, D, y, \
+  k_decode_window_step<T, NN><<<grid, 256, 0, st>>>(state, win_x, win_dt, win_B, W, pos, x, dt, A, B, C, D, y, \
                                                        d)
   switch (d.N) {
     case 16: SSD_WSTEP(16); break;
