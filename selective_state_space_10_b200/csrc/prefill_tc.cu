@@ -111,7 +111,9 @@ k_chunk_state_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
                  float *__restrict__ tab, float *__restrict__ cdecay, float *__restrict__ states, int *err, Dims d, int Q,
                  int nc, int kb, int nhb) {
   extern __shared__ uint8_t smem_raw[];
-  uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // 1024-byte aligned, and derived from the shared array itself (no integer round trip),
+  // so that the compiler keeps every access through it in the shared address space
+  uint8_t *base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   K1Misc *ms = reinterpret_cast<K1Misc *>(base + K1Smem::misc(Q));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -542,7 +544,9 @@ k_chunk_scan_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
                 const __grid_constant__ CUtensorMap tm_y, const float *__restrict__ tab, int *err, Dims d, int Q, int nc,
                 int kb0, int nhb0, int kb1, int nhb1) {
   extern __shared__ uint8_t smem_raw[];
-  uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // 1024-byte aligned, and derived from the shared array itself (no integer round trip),
+  // so that the compiler keeps every access through it in the shared address space
+  uint8_t *base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   K3Misc *ms = reinterpret_cast<K3Misc *>(base + K3Smem::misc);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
