@@ -19,6 +19,7 @@
 // place.
 #include "common.cuh"
 #include "kernels.h"
+#include "sm100.cuh"
 
 namespace ssd {
 
@@ -104,6 +105,58 @@ k_frontend(const T *__restrict__ xbc, const float *__restrict__ w, const float *
   constexpr int kFeTokens = fe_tokens<T>();
   const int t0 = blockIdx.x * kFeTokens, bi = blockIdx.z;
   const int t1 = min(t0 + kFeTokens, d.L);
+  // Stage this CTA's inputs -- rows t0-3 .. t1-1 of its 256 * V channels -- in shared
+  // memory with asynchronous copies (nothing held in registers while they fly): with 4
+  // channels a thread, one bulk copy per row by one thread, completing on an mbarrier;
+  // otherwise a cp.async per thread and row.  Rows before the sequence come from the conv
+  // state or are zero.
+  __shared__ __align__(16) T tile[3 + kFeTokens][256 * V];
+  __shared__ uint64_t rows_full;
+  const int tl = threadIdx.x * V;  // this thread's first channel within the tile
+  const bool active = c < CH;
+  const int cbase = blockIdx.y * 256 * V, nch = min(256 * V, CH - cbase);
+  const bool bulk = V == 4 && (nch * (int)sizeof(T)) % 16 == 0 && ((size_t)CH * sizeof(T)) % 16 == 0 &&
+                    reinterpret_cast<uintptr_t>(xbc) % 16 == 0;
+  const T *uc = xbc + (size_t)bi * d.L * CH + c;
+  if (bulk) {
+    if (threadIdx.x == 0) {
+      sm100::mbar_init(&rows_full, 1);
+      sm100::mbar_fence_init();
+      uint32_t bytes = 0;
+      for (int j = 0; j < 3 + kFeTokens; ++j) {
+        const int t = t0 - 3 + j;
+        if (t >= 0 && t < t1) bytes += (uint32_t)nch * sizeof(T);
+      }
+      sm100::mbar_arrive_expect_tx(&rows_full, bytes);
+      for (int j = 0; j < 3 + kFeTokens; ++j) {
+        const int t = t0 - 3 + j;
+        if (t >= 0 && t < t1)
+          sm100::bulk_load(&tile[j][0], xbc + ((size_t)bi * d.L + t) * CH + cbase, (uint32_t)nch * sizeof(T),
+                           &rows_full);
+      }
+    }
+    __syncthreads();  // the barrier is initialised before any thread waits on it
+  } else if (active) {
+#pragma unroll
+    for (int j = 0; j < 3 + kFeTokens; ++j) {
+      const int t = t0 - 3 + j;
+      if (t >= 0 && t < t1) {
+        if constexpr (sizeof(T) * V >= 4)
+          cp_async<sizeof(T) * V>(&tile[j][tl], uc + (size_t)t * CH);
+        else
+          tile[j][tl] = uc[(size_t)t * CH];  // the scalar bf16 fallback (2 bytes)
+      }
+    }
+  }
+  if (active)
+#pragma unroll
+    for (int j = 0; j < 3; ++j) {
+      const int t = t0 - 3 + j;
+      if (t < 0)
+#pragma unroll
+        for (int q = 0; q < V; ++q)
+          tile[j][tl + q] = from_f32<T>(state_in ? state_in[((size_t)bi * 3 + (3 + t)) * CH + c + q] : 0.f);
+    }
   if (blockIdx.y == 0) {  // dt for this run of tokens (all loads issued before any use)
     for (int h = threadIdx.x; h < d.H; h += blockDim.x) {
       const float bh = dt_bias[h];
@@ -116,29 +169,6 @@ k_frontend(const T *__restrict__ xbc, const float *__restrict__ w, const float *
         if (t0 + j < t1) dt[((size_t)bi * d.L + t0 + j) * d.H + h] = softplus_f(z[j] + bh);
     }
   }
-  // Stage this CTA's inputs -- rows t0-3 .. t1-1 of its 256 * V channels -- in shared
-  // memory with asynchronous copies (nothing held in registers while they fly); rows
-  // before the sequence come from the conv state or are zero.
-  __shared__ __align__(16) T tile[3 + kFeTokens][256 * V];
-  const int tl = threadIdx.x * V;  // this thread's first channel within the tile
-  const bool active = c < CH;
-  if (active) {
-    const T *uc = xbc + (size_t)bi * d.L * CH + c;
-#pragma unroll
-    for (int j = 0; j < 3 + kFeTokens; ++j) {
-      const int t = t0 - 3 + j;
-      if (t >= 0 && t < t1) {
-        if constexpr (sizeof(T) * V >= 4)
-          cp_async<sizeof(T) * V>(&tile[j][tl], uc + (size_t)t * CH);
-        else
-          tile[j][tl] = uc[(size_t)t * CH];  // the scalar bf16 fallback (2 bytes)
-      } else if (t < 0) {
-#pragma unroll
-        for (int q = 0; q < V; ++q)
-          tile[j][tl + q] = from_f32<T>(state_in ? state_in[((size_t)bi * 3 + (3 + t)) * CH + c + q] : 0.f);
-      }
-    }
-  }
   // the filters while the copies fly
   float4 wc[V];
   float bc[V];
@@ -147,9 +177,10 @@ k_frontend(const T *__restrict__ xbc, const float *__restrict__ w, const float *
     wc[q] = active ? *reinterpret_cast<const float4 *>(w + (size_t)(c + q) * 4) : make_float4(0.f, 0.f, 0.f, 0.f);
     bc[q] = (active && bias) ? bias[c + q] : 0.f;
   }
-  cp_async_wait_all();
+  // the copies have landed (bounded wait: after 2 s the CTA gives up, its outputs undefined)
+  const bool landed = bulk ? sm100::mbar_wait_drain(&rows_full, 0) : (cp_async_wait_all(), true);
   __syncthreads();
-  if (!active) return;
+  if (!active || !landed) return;
   T *dst;
   size_t stride;
   if (c < HP) {
