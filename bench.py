@@ -443,25 +443,37 @@ def prefill_leg(args, dev, rank, world, peaks, sampler):
                    "parallelism": f"{world} GPU(s), one independent sequence per GPU, no collective"},
     }
     # End to end through the C ABI's host-buffer call: pinned host inputs -> device copies ->
-    # prefill -> y and final state -> pinned host, all enqueued by ssd_prefill_host.
+    # prefill -> y and final state -> pinned host, all enqueued by ssd_prefill_host.  Each step
+    # is an independent sequence, so consecutive steps alternate between two streams (each with
+    # its own device buffer and host outputs): one step's y copy back overlaps the next step's
+    # input copies and kernels, as two requests would in a server.
     host = {k: v.cpu().pin_memory() for k, v in t.items()}
-    y_h = torch.empty(y.shape, dtype=y.dtype, pin_memory=True)
-    fs_h = torch.empty(fs.shape, dtype=fs.dtype, pin_memory=True)
-    hbuf = torch.empty(ssd.prefill_host_buffer_size(dims, dtype, w.chunk), dtype=torch.uint8, device=dev)
     h2d = sum(v.numel() * v.element_size() for v in host.values())
     d2h = y.numel() * 4 + fs.numel() * 4
     ke = max(3, min(K, 20))
+    lanes = [torch.cuda.Stream(dev) for _ in range(2)]
+    lane_y = [torch.empty(y.shape, dtype=y.dtype, pin_memory=True) for _ in lanes]
+    lane_fs = [torch.empty(fs.shape, dtype=fs.dtype, pin_memory=True) for _ in lanes]
+    lane_buf = [torch.empty(ssd.prefill_host_buffer_size(dims, dtype, w.chunk), dtype=torch.uint8, device=dev)
+                for _ in lanes]
 
-    def e2e_step():
-        ssd.prefill_host(**host, chunk=w.chunk, y=y_h, final_state=fs_h, device_buffer=hbuf, stream=stream)
-    for _ in range(2):
-        e2e_step()
+    def e2e_step(k):
+        j = k % len(lanes)
+        ssd.prefill_host(**host, chunk=w.chunk, y=lane_y[j], final_state=lane_fs[j], device_buffer=lane_buf[j],
+                         stream=lanes[j])
+    torch.cuda.synchronize(dev)
+    for k in range(2):
+        e2e_step(k)
     torch.cuda.synchronize(dev)
     barrier(world, dev)
     a, b = mk(), mk()
     a.record(stream)
-    for _ in range(ke):
-        e2e_step()
+    for s_ in lanes:
+        s_.wait_event(a)
+    for k in range(ke):
+        e2e_step(k)
+    for s_ in lanes:
+        stream.wait_stream(s_)
     b.record(stream)
     torch.cuda.synchronize(dev)
     barrier(world, dev)
@@ -469,7 +481,7 @@ def prefill_leg(args, dev, rank, world, peaks, sampler):
     res["e2e"] = {"value": world * tokens * ke / (e2e_ms / 1e3), "unit": "tokens/s", "steps": ke,
                   "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                   "path": "ssd_prefill_host (C ABI): pinned host x, dt, A, B, C, D -> device copies -> prefill -> "
-                          "y, final_state -> pinned host"}
+                          "y, final_state -> pinned host; consecutive sequences on two streams"}
     return res
 
 
@@ -626,34 +638,63 @@ def decode_leg(args, dev, rank, world, peaks, sampler):
                    "input_dtype": "bf16", "state_dtype": "f32", "y_dtype": "f32",
                    "l2": "state (671 MB) larger than L2; no flush"},
     }
-    # End to end: per step, the step's inputs from pinned host memory and y back.
+    # End to end: per step, the step's inputs from pinned host memory and y back.  The steps
+    # are sequential (each continues from the state the one before wrote), but their copies
+    # need not wait for the compute: step k+1's inputs go up on one copy stream while step k
+    # runs, and step k's y comes back on another while step k+1 runs (device inputs and y
+    # double-buffered, the reuse of each buffer ordered by events).
     ke = min(nsteps, 64)
     hx = xs[:ke].cpu().pin_memory()
     hdt = dts[:ke].cpu().pin_memory()
     hB = Bs[:ke].cpu().pin_memory()
     hC = Cs[:ke].cpu().pin_memory()
     y_h = torch.empty((ke,) + tuple(y.shape), dtype=y.dtype, pin_memory=True)
-    dx, ddt, dB, dC = (torch.empty_like(xs[0]), torch.empty_like(dts[0]), torch.empty_like(Bs[0]),
-                       torch.empty_like(Cs[0]))
+    nbuf = 2
+    dx = [torch.empty_like(xs[0]) for _ in range(nbuf)]
+    ddt = [torch.empty_like(dts[0]) for _ in range(nbuf)]
+    dB = [torch.empty_like(Bs[0]) for _ in range(nbuf)]
+    dC = [torch.empty_like(Cs[0]) for _ in range(nbuf)]
+    dy = [torch.empty_like(y) for _ in range(nbuf)]
+    up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev_in = [torch.cuda.Event() for _ in range(ke)]
+    ev_done = [torch.cuda.Event() for _ in range(ke)]
+    ev_out = [torch.cuda.Event() for _ in range(ke)]
     torch.cuda.synchronize(dev)
     barrier(world, dev)
     a, e = mk(), mk()
     a.record(stream)
+    up.wait_event(a)
+    down.wait_event(a)
     for k in range(ke):
-        dx.copy_(hx[k], non_blocking=True)
-        ddt.copy_(hdt[k], non_blocking=True)
-        dB.copy_(hB[k], non_blocking=True)
-        dC.copy_(hC[k], non_blocking=True)
-        ssd.decode_step(state, dx, ddt, A, dB, dC, D, y=y, stream=stream)
-        y_h[k].copy_(y, non_blocking=True)
+        j = k % nbuf
+        with torch.cuda.stream(up):
+            if k >= nbuf:
+                up.wait_event(ev_done[k - nbuf])  # the step that last read these inputs has run
+            dx[j].copy_(hx[k], non_blocking=True)
+            ddt[j].copy_(hdt[k], non_blocking=True)
+            dB[j].copy_(hB[k], non_blocking=True)
+            dC[j].copy_(hC[k], non_blocking=True)
+            ev_in[k].record(up)
+        stream.wait_event(ev_in[k])
+        if k >= nbuf:
+            stream.wait_event(ev_out[k - nbuf])  # this y buffer's last copy back has finished
+        ssd.decode_step(state, dx[j], ddt[j], A, dB[j], dC[j], D, y=dy[j], stream=stream)
+        ev_done[k].record(stream)
+        with torch.cuda.stream(down):
+            down.wait_event(ev_done[k])
+            y_h[k].copy_(dy[j], non_blocking=True)
+            ev_out[k].record(down)
+    stream.wait_stream(down)
     e.record(stream)
     torch.cuda.synchronize(dev)
     barrier(world, dev)
     e2e_ms = max_over_ranks(a.elapsed_time(e), world, dev)
     res["e2e"] = {"value": world * ke / (e2e_ms / 1e3), "unit": "steps/s", "steps": ke,
-                  "h2d_bytes_per_step": dx.numel() * 2 + ddt.numel() * 4 + dB.numel() * 2 + dC.numel() * 2,
+                  "h2d_bytes_per_step": dx[0].numel() * 2 + ddt[0].numel() * 4 + dB[0].numel() * 2
+                  + dC[0].numel() * 2,
                   "d2h_bytes_per_step": y.numel() * 4,
-                  "path": "pinned host x, dt, B, C -> device -> ssd_decode_step -> y -> pinned host"}
+                  "path": "pinned host x, dt, B, C -> device -> ssd_decode_step -> y -> pinned host; inputs up "
+                          "and y back on two copy streams, overlapping the neighbouring steps"}
     return res
 
 
