@@ -478,7 +478,12 @@ def prefill_leg(args, dev, rank, world, peaks, sampler):
     torch.cuda.synchronize(dev)
     barrier(world, dev)
     e2e_ms = max_over_ranks(a.elapsed_time(b), world, dev)
+    call()  # the device-only call on the same inputs: the host outputs must equal it bit for bit
+    torch.cuda.synchronize(dev)
+    y_ref, fs_ref = y.cpu(), fs.cpu()
+    same = all(torch.equal(yl, y_ref) and torch.equal(fl, fs_ref) for yl, fl in zip(lane_y, lane_fs))
     res["e2e"] = {"value": world * tokens * ke / (e2e_ms / 1e3), "unit": "tokens/s", "steps": ke,
+                  "outputs_match_device_call": bool(same),
                   "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                   "path": "ssd_prefill_host (C ABI): pinned host x, dt, A, B, C, D -> device copies -> prefill -> "
                           "y, final_state -> pinned host; consecutive sequences on two streams"}
@@ -656,6 +661,7 @@ def decode_leg(args, dev, rank, world, peaks, sampler):
     dC = [torch.empty_like(Cs[0]) for _ in range(nbuf)]
     dy = [torch.empty_like(y) for _ in range(nbuf)]
     up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    snapshot = state.clone()  # to replay the same steps in order afterwards, as a check
     ev_in = [torch.cuda.Event() for _ in range(ke)]
     ev_done = [torch.cuda.Event() for _ in range(ke)]
     ev_out = [torch.cuda.Event() for _ in range(ke)]
@@ -689,7 +695,16 @@ def decode_leg(args, dev, rank, world, peaks, sampler):
     torch.cuda.synchronize(dev)
     barrier(world, dev)
     e2e_ms = max_over_ranks(a.elapsed_time(e), world, dev)
+    # the overlapped copies must not change what the steps compute: replay them in order on
+    # one stream from the same state and compare every y bit for bit
+    state.copy_(snapshot)
+    del snapshot
+    same = True
+    for k in range(ke):
+        yk = ssd.decode_step(state, xs[k], dts[k], A, Bs[k], Cs[k], D, stream=stream)
+        same = same and torch.equal(yk.cpu(), y_h[k])
     res["e2e"] = {"value": world * ke / (e2e_ms / 1e3), "unit": "steps/s", "steps": ke,
+                  "outputs_match_in_order_steps": bool(same),
                   "h2d_bytes_per_step": dx[0].numel() * 2 + ddt[0].numel() * 4 + dB[0].numel() * 2
                   + dC[0].numel() * 2,
                   "d2h_bytes_per_step": y.numel() * 4,

@@ -260,6 +260,86 @@ def test_prefill_host_equals_the_device_call(ssd, dtype, shape):
         assert torch.equal(yh, y.cpu()) and torch.equal(fsh, fs.cpu())
 
 
+def test_prefill_host_on_two_streams_matches_each_device_call(ssd):
+    """Independent sequences alternating between two streams, each stream with its own
+    device buffer, so that one call's copies back overlap the next call's copies in and
+    kernels: every sequence's host y and final state equal its own device call bit for bit."""
+    Q = 256
+    seqs = [to_device(inputs.sequence(1, 700, 4, 64, 128, 1, "bf16", seed=500 + i)) for i in range(4)]
+    refs = []
+    for t in seqs:
+        y, fs = ssd.prefill(**t, chunk=Q)
+        refs.append((y.cpu(), fs.cpu()))
+    dims = ssd.dims_of_prefill(seqs[0]["x"], seqs[0]["B"])
+    lanes = [torch.cuda.Stream() for _ in range(2)]
+    bufs = [torch.empty(ssd.prefill_host_buffer_size(dims, ssd.BF16, Q), dtype=torch.uint8, device="cuda")
+            for _ in lanes]
+    hosts = [{k: v.cpu().pin_memory() for k, v in t.items()} for t in seqs]
+    torch.cuda.synchronize()
+    outs = [ssd.prefill_host(**h, chunk=Q, device_buffer=bufs[i % 2], stream=lanes[i % 2])
+            for i, h in enumerate(hosts)]
+    torch.cuda.synchronize()
+    for (yh, fsh), (y, fs) in zip(outs, refs):
+        assert torch.equal(yh, y) and torch.equal(fsh, fs)
+
+
+def test_decode_with_copies_on_side_streams_matches_in_order_steps(ssd):
+    """Decode steps in order on the compute stream while each step's inputs go up on one
+    copy stream and its y comes back on another (device inputs and y double-buffered, their
+    reuse ordered by events): every y and the final state equal those of the same steps run
+    plainly on one stream, bit for bit."""
+    b, H, P, N, G, steps = 8, 6, 64, 128, 1, 12
+    g = torch.Generator().manual_seed(91)
+    hx = torch.randn((steps, b, H, P), generator=g).bfloat16().pin_memory()
+    hdt = (torch.rand((steps, b, H), generator=g) * 0.1 + 1e-3).pin_memory()
+    hB = (torch.randn((steps, b, G, N), generator=g) / N ** 0.5).bfloat16().pin_memory()
+    hC = (torch.randn((steps, b, G, N), generator=g) / N ** 0.5).bfloat16().pin_memory()
+    A = (-torch.exp(torch.rand((H,), generator=g) * np.log(16.0))).cuda()
+    D = torch.randn((H,), generator=g).cuda()
+    state0 = (torch.randn((b, H, P, N), generator=g) * 0.1).cuda()
+
+    state = state0.clone()
+    ref = []
+    for k in range(steps):
+        ref.append(ssd.decode_step(state, hx[k].cuda(), hdt[k].cuda(), A, hB[k].cuda(), hC[k].cuda(), D).cpu())
+    ref_state = state.cpu()
+
+    state = state0.clone()
+    main = torch.cuda.current_stream()
+    up, down = torch.cuda.Stream(), torch.cuda.Stream()
+    dx = [torch.empty((b, H, P), dtype=torch.bfloat16, device="cuda") for _ in range(2)]
+    ddt = [torch.empty((b, H), device="cuda") for _ in range(2)]
+    dB = [torch.empty((b, G, N), dtype=torch.bfloat16, device="cuda") for _ in range(2)]
+    dC = [torch.empty((b, G, N), dtype=torch.bfloat16, device="cuda") for _ in range(2)]
+    dy = [torch.empty((b, H, P), device="cuda") for _ in range(2)]
+    y_h = torch.empty((steps, b, H, P), pin_memory=True)
+    ev_in, ev_done, ev_out = ([torch.cuda.Event() for _ in range(steps)] for _ in range(3))
+    torch.cuda.synchronize()
+    for k in range(steps):
+        j = k % 2
+        with torch.cuda.stream(up):
+            if k >= 2:
+                up.wait_event(ev_done[k - 2])
+            dx[j].copy_(hx[k], non_blocking=True)
+            ddt[j].copy_(hdt[k], non_blocking=True)
+            dB[j].copy_(hB[k], non_blocking=True)
+            dC[j].copy_(hC[k], non_blocking=True)
+            ev_in[k].record(up)
+        main.wait_event(ev_in[k])
+        if k >= 2:
+            main.wait_event(ev_out[k - 2])
+        ssd.decode_step(state, dx[j], ddt[j], A, dB[j], dC[j], D, y=dy[j], stream=main)
+        ev_done[k].record(main)
+        with torch.cuda.stream(down):
+            down.wait_event(ev_done[k])
+            y_h[k].copy_(dy[j], non_blocking=True)
+            ev_out[k].record(down)
+    torch.cuda.synchronize()
+    for k in range(steps):
+        assert torch.equal(y_h[k], ref[k]), f"step {k}"
+    assert torch.equal(state.cpu(), ref_state)
+
+
 @pytest.mark.parametrize("L", [500, 400])
 def test_wide_decay_ranges_take_every_factorisation(ssd, L):
     """The tensor-core chunk scan factorises a tile's decays three ways: one reference token
