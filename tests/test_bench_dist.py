@@ -77,3 +77,26 @@ def test_kernel_work_is_below_the_ridge_for_the_tensor_core_kernels():
         kind, nbytes, _, flops = bench.kernel_work(name, w, w.chunk)
         assert kind == "hbm" and nbytes > 0
         assert flops / nbytes < 1657.6e12 / 6539.2e9  # arithmetic intensity below the ridge
+
+
+def test_committed_traffic_counters_follow_the_kernel_sources(tmp_path, monkeypatch):
+    """The roofline's `traffic` comes from a committed ncu summary only while the code of the
+    kernel's sources is the code that was profiled: the summaries in profiles/ match the
+    current sources, a changed statement voids them, a changed comment does not."""
+    for kernel in ("chunk_scan_tc", "chunk_state_tc", "state_passing_bf16", "decode_step"):
+        wl = "mamba2_2.7b_decode_b256" if kernel == "decode_step" else "mamba2_2.7b_prefill"
+        assert bench.profile_traffic(kernel, wl) > 0, kernel
+    assert bench.profile_traffic("chunk_scan_tc", "no_such_workload") is None
+
+    src = tmp_path / "k.cu"
+    src.write_text("__global__ void k(float *p) { p[0] = 1.f; }  // one\n")
+    (tmp_path / "profiles").mkdir()
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    digest = bench.source_digest(["k.cu"])
+    (tmp_path / "profiles" / "k.w.txt").write_text(
+        f"# summary\ntraffic_bytes_per_launch = 1234\nsources = k.cu\nsources_sha256 = {digest}\n")
+    assert bench.profile_traffic("k", "w") == 1234.0
+    src.write_text("__global__ void k(float *p) {\n  p[0] = 1.f;  /* two */\n}\n")
+    assert bench.profile_traffic("k", "w") == 1234.0      # comments and layout only
+    src.write_text("__global__ void k(float *p) { p[0] = 2.f; }\n")
+    assert bench.profile_traffic("k", "w") is None        # the code changed
