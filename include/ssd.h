@@ -33,8 +33,12 @@
  *
  * Conventions of every call:
  *   - All array pointers are DEVICE pointers on the current CUDA device, owned by the
- *     caller.  libssd never allocates, frees or keeps device memory, and keeps no state
- *     between calls.  A pointer may be NULL only if its array has zero elements.
+ *     caller.  libssd never allocates or frees device memory, and keeps no state between
+ *     calls that changes a result.  The one exception is ssd_prefill_noalloc: its scratch
+ *     is a fixed device array inside the library (held on a device from its first use
+ *     there), whose address it caches per CUDA context.  Host-side caches of encoded
+ *     tensor maps and of per-device kernel attributes only save set-up time.  A pointer
+ *     may be NULL only if its array has zero elements.
  *   - x, B, C, y, state, final_state and workspace must be 16-byte aligned; dt, A and D
  *     4-byte aligned.
  *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy default
@@ -68,7 +72,7 @@ typedef enum {
   SSD_ERR_UNSUPPORTED = 2, /* valid but outside the compiled shape set (see below)        */
   SSD_ERR_WORKSPACE = 3,   /* workspace NULL or smaller than ssd_prefill_workspace_size()  */
   SSD_ERR_CUDA = 4,        /* a CUDA runtime call or kernel launch failed                  */
-  SSD_ERR_TIMEOUT = 5      /* reserved for bounded device-side waits; not returned today    */
+  SSD_ERR_TIMEOUT = 5      /* a bounded device-side wait expired (ssd_prefill_device_status) */
 } ssd_status;
 
 typedef enum {
@@ -196,9 +200,13 @@ SSD_API ssd_status ssd_prefill_device_status(const void *workspace, size_t works
  *
  *   - Allocates nothing: no cudaMalloc, cudaFree or allocating library routine.  The
  *     array is held on a device, until the process exits, from the first call on it.
- *   - The first call on a device, with that device current, looks up the array's device
- *     address (cudaGetSymbolAddress) and caches it; make that first call before any
- *     stream capture.
+ *   - The first call in a CUDA context (on a device, with its context current) looks
+ *     up the array's device address there (cudaGetSymbolAddress) and caches it under the
+ *     context's unique id; make that first call before any stream capture.  A new context
+ *     (after cudaDeviceReset, or another one the caller made current) gets its own
+ *     look-up, never a stale address.
+ *   - A bounded device wait that expired is reported by
+ *     ssd_prefill_noalloc_device_status, which reads the array's error word.
  *   - Every call shares the one array: calls whose executions overlap on the GPU (other
  *     streams, other host threads without ordering) race and give undefined results.
  *     Order them on one stream or synchronise between them.
@@ -227,6 +235,15 @@ SSD_API ssd_status ssd_wait_selftest(void *workspace, size_t workspace_bytes, ui
 
 /* Size in bytes of the fixed scratch array ssd_prefill_noalloc uses (32 MiB). */
 SSD_API size_t ssd_prefill_noalloc_max_workspace(void);
+
+/*
+ * ssd_prefill_device_status for ssd_prefill_noalloc, whose callers hold no workspace:
+ * waits for `stream`, then reads the error word of the library's scratch array in the
+ * current context.  SSD_ERR_TIMEOUT if a bounded wait of the last noalloc prefill on it
+ * expired (y and final_state are then undefined), SSD_OK otherwise; SSD_ERR_CUDA if the
+ * look-up, the copy or the synchronisation fails.  Allocates nothing; blocks the host.
+ */
+SSD_API ssd_status ssd_prefill_noalloc_device_status(ssd_stream_t stream);
 
 /*
  * The prefill end to end, with HOST arrays: copies x, dt, A, B, C and D to the device,

@@ -47,6 +47,7 @@
 #include <stddef.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <functional>
 #include <map>
@@ -129,7 +130,6 @@ k_chunk_state_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
   const int nh = min(kb, d.hpg - hb * kb);
   const int t0 = c * Q;
   const int valid = min(Q, d.L - t0);
-  grid_dep_launch();  // state passing may be scheduled now; it waits for this grid's results
 
   if (threadIdx.x == 0) {
     mbar_init(&ms->b_full, 1);
@@ -155,6 +155,17 @@ k_chunk_state_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
   tc_fence_after();
   const uint32_t tmem = ms->tmem;
   volatile int *abort_flag = &ms->abort_flag;
+  // Launched as a programmatic dependent of whatever the stream ran before: the set-up
+  // above overlaps that kernel's tail, and nothing global is read or written before it has
+  // completed (it may have produced x, dt, B, or still be reading this workspace).
+  grid_dep_wait();
+  // Only now may state passing be scheduled (it waits for this grid's results).  Its own
+  // dependent, the chunk scan, reads x, B and C without waiting: by then the kernel that
+  // produced them has completed.
+  grid_dep_launch();
+  // The device error word starts each prefill at zero.  A kernel of this prefill raises it
+  // only after a bounded wait of 2 s has expired, long after this store.
+  if (blockIdx.x == 0 && threadIdx.x == 0) *err = 0;
 
   if (warp == 0) {
     // ------------------------------------------------------------- TMA producer
@@ -337,7 +348,8 @@ k_chunk_state_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
       const bool ok = mbar_wait(&ms->acc_full[a], (k >> 1) & 1, abort_flag, err);
       tc_fence_after();
       if (ok) {
-        float *out = states + (((size_t)bi * nc + c) * d.H + h) * (size_t)(TP * TN) + n;
+        // S in the layout of the entering states: [n / 64][p][n % 64] per (batch, chunk, head)
+        float *out = states + (((size_t)bi * nc + c) * d.H + h) * (size_t)(TP * TN) + (n >> 6) * (TP * 64) + (n & 63);
 #pragma unroll
         for (int cg = 0; cg < 2; ++cg) {
           float vh[32], vl[32];
@@ -345,7 +357,7 @@ k_chunk_state_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
           tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(a * 2 * TP + TP + cg * 32), vl);
           tmem_ld_wait();
 #pragma unroll
-          for (int j = 0; j < 32; ++j) out[(size_t)(cg * 32 + j) * TN] = vh[j] + vl[j];
+          for (int j = 0; j < 32; ++j) out[(size_t)(cg * 32 + j) * 64] = vh[j] + vl[j];
         }
       }
       tc_fence_before();
@@ -381,6 +393,9 @@ __device__ __forceinline__ void cp_async16(void *dst, const void *src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
 }
 
+// kExport: also store the state after every chunk (cstates non-NULL); a separate
+// instantiation, so that the plain prefill's kernel holds no pointer for it.
+template <bool kExport>
 __global__ void __launch_bounds__(K2_THREADS, 4)
 k_state_passing_bf16(const float *__restrict__ states, const float *__restrict__ cdecay,
                      __nv_bfloat16 *__restrict__ hprev, const float *init, float *final_state,
@@ -393,13 +408,19 @@ k_state_passing_bf16(const float *__restrict__ states, const float *__restrict__
   if (e4 >= PN4) return;
   const int h = blockIdx.x % d.H, bi = blockIdx.x / d.H;
   const size_t cstride = (size_t)d.H * PN4;  // float4s between consecutive chunks
+  // The chunk states S (fp32) and the bf16 entering states of a (batch, chunk, head) share
+  // one layout: the two 64-wide halves of d_state, [n / 64][p][n % 64] (d_state = 128), so
+  // that the chunk-scan kernel fetches an entering state with one box.  e4 indexes four
+  // consecutive elements of that layout; e4o is the same four elements in a [p][n] state.
   const size_t off0 = ((size_t)bi * nc * d.H + h) * PN4 + e4;
   const float4 *sp = reinterpret_cast<const float4 *>(states) + off0;
   uint2 *hp = reinterpret_cast<uint2 *>(hprev) + off0;
+  const int half = (4 * e4) / (d.P * 64), rem = 4 * e4 - half * d.P * 64;
+  const int e4o = ((rem >> 6) * d.N + half * 64 + (rem & 63)) >> 2;
   const float *dec = cdecay + ((size_t)bi * d.H + h) * nc;
-  const size_t own4 = ((size_t)bi * d.H + h) * PN4 + e4;  // this element in a [b][H][P][N] state
+  const size_t own4 = ((size_t)bi * d.H + h) * PN4 + e4o;  // this element in a [b][H][P][N] state
   float4 hs = init ? reinterpret_cast<const float4 *>(init)[own4] : make_float4(0.f, 0.f, 0.f, 0.f);
-  float4 *cs = cstates ? reinterpret_cast<float4 *>(cstates) + off0 : nullptr;
+  float4 *cs = kExport ? reinterpret_cast<float4 *>(cstates) + ((size_t)bi * nc * d.H + h) * PN4 + e4o : nullptr;
   float4 *stage = k2_stage + threadIdx.x;
   auto step = [&](int c, const float4 &sv) {
     const float dc = __ldg(dec + c);
@@ -408,7 +429,7 @@ k_state_passing_bf16(const float *__restrict__ states, const float *__restrict__
     hs.y = fmaf(dc, hs.y, sv.y);
     hs.z = fmaf(dc, hs.z, sv.z);
     hs.w = fmaf(dc, hs.w, sv.w);
-    if (cs) cs[(size_t)c * cstride] = hs;  // state after chunk c
+    if (kExport) cs[(size_t)c * cstride] = hs;  // state after chunk c
   };
   for (int c0 = 0; c0 < nc; c0 += K2_ROUND) {
     // issue the whole round: chunks c0 .. c0+7 into registers, c0+8 .. c0+15 into shared memory
@@ -455,8 +476,9 @@ k_state_passing_bf16(const float *__restrict__ states, const float *__restrict__
 // x row anyway, store D x_t / u_t into the intra-chunk accumulator before the MMA adds
 // W X' onto it; the output warps then only combine the two accumulators and hand each
 // [32 rows][32 channels] tile of y to a TMA store.
-constexpr int K3_THREADS = 672;  // warp 0 TMA, 1 MMA (G, inter), 2-5 and 17-20 W/x scaling, 6-13 output,
-                                 // 14 decay-table loads, 15 MMA (intra, source block 0), 16 MMA (intra, block 1)
+constexpr int K3_THREADS = 704;  // warp 0 TMA (C, B, x), 1 MMA (G, inter), 2-5 and 17-20 W/x scaling, 6-13 output,
+                                 // 14 decay-table loads, 15 MMA (intra, source block 0), 16 MMA (intra, block 1),
+                                 // 21 TMA (entering states)
 constexpr int K3_CUMBUF = 4;
 constexpr int K3_MAXSLOTS = 5;
 constexpr float kSteepLog2 = 100.f;
@@ -485,7 +507,7 @@ static_assert(K3Smem::ring % 1024 == 0 && K3Smem::bm(1) % 1024 == 0 && K3Smem::b
 
 struct K3Misc {
   uint64_t cb_full, g_full, w_ready;
-  uint64_t x_full[K3_MAXSLOTS], ops_ready[K3_MAXSLOTS], x_free[K3_MAXSLOTS];
+  uint64_t x_full[K3_MAXSLOTS], h_full[K3_MAXSLOTS], ops_ready[K3_MAXSLOTS], x_free[K3_MAXSLOTS];
   uint64_t acc_full[2], acc_free[2];
   uint64_t tab_full[K3_CUMBUF], cum_free[K3_CUMBUF];
   uint32_t tmem;
@@ -539,7 +561,8 @@ constexpr uint32_t K3_TM_WB = 0, K3_TM_BUF = 128, K3_BUF_COLS = 192;
 __device__ __forceinline__ uint32_t k3_buf(int a) { return K3_TM_BUF + K3_BUF_COLS * (uint32_t)a; }
 
 __global__ void __launch_bounds__(K3_THREADS, 1)
-k_chunk_scan_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_C,
+k_chunk_scan_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_x2,
+                const __grid_constant__ CUtensorMap tm_C,
                 const __grid_constant__ CUtensorMap tm_B, const __grid_constant__ CUtensorMap tm_h,
                 const __grid_constant__ CUtensorMap tm_y, const float *__restrict__ tab, int *err, Dims d, int Q, int nc,
                 int kb0, int nhb0, int kb1, int nhb1) {
@@ -570,6 +593,7 @@ k_chunk_scan_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
   const int nblk = ti + 1;        // source blocks j = 0..ti
   const int NS = K3Smem::slots(nblk);
   const uint32_t SB = K3Smem::slot_bytes(nblk);
+  const uint32_t SBX = (uint32_t)nblk * 16384u;  // the slot's x part; the entering state follows it
 
   if (threadIdx.x == 0) {
     mbar_init(&ms->cb_full, 1);
@@ -577,6 +601,7 @@ k_chunk_scan_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
     mbar_init(&ms->w_ready, 1);
     for (int s = 0; s < K3_MAXSLOTS; ++s) {
       mbar_init(&ms->x_full[s], 1);
+      mbar_init(&ms->h_full[s], 1);
       mbar_init(&ms->ops_ready[s], 1);
       mbar_init(&ms->x_free[s], 3);  // commits of the three MMA issuers
     }
@@ -604,10 +629,14 @@ k_chunk_scan_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
   if (warp == 0) {
     // ------------------------------------------------------------- TMA producer
     if (lane == 0) {
-      tma_prefetch_desc(&tm_x);
+      // x of a head: one box of the tile's 128 * nblk rows (the second row tile's two
+      // source blocks are consecutive rows).  The entering states come from warp 21: a
+      // thread completes about one TMA box per half microsecond however many it has in
+      // flight, so the per-head boxes are spread over two issuing threads.
+      const CUtensorMap *xm = nblk == 2 ? &tm_x2 : &tm_x;
+      tma_prefetch_desc(xm);
       tma_prefetch_desc(&tm_C);
       tma_prefetch_desc(&tm_B);
-      tma_prefetch_desc(&tm_h);
       tma_prefetch_desc(&tm_y);
       const uint32_t bmo = K3Smem::bm(nblk);
       mbar_arrive_expect_tx(&ms->cb_full, 32768u + (uint32_t)nblk * 32768u);
@@ -622,31 +651,22 @@ k_chunk_scan_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
       // overlaps the B rows is filled only once G has been formed.
       int pre = 0;
       while (pre < min(nh, NS) && K3Smem::slot(nblk, pre) + SB <= bmo) {
-        mbar_arrive_expect_tx(&ms->x_full[pre], SB);
-        for (int jj = 0; jj < nblk; ++jj)
-          tma_load_3d(base + K3Smem::slot(nblk, pre) + jj * 16384u, &tm_x, &ms->x_full[pre], (h0 + pre) * TP,
-                      t0 + 128 * jj, bi);
+        mbar_arrive_expect_tx(&ms->x_full[pre], SBX);
+        tma_load_3d(base + K3Smem::slot(nblk, pre), xm, &ms->x_full[pre], (h0 + pre) * TP, t0, bi);
         ++pre;
       }
-      grid_dep_wait();
       bool g_seen = false;
-      int issued = 0;
-      for (int k = 0; k < nh; ++k) {
+      int issued = pre;
+      for (int k = pre; k < nh; ++k) {
         const int s = k % NS, u = k / NS, h = h0 + k;
         const uint32_t so = K3Smem::slot(nblk, s);
-        if (k >= pre) {
-          if (k >= NS) {
-            if (!mbar_wait(&ms->x_free[s], (u - 1) & 1, abort_flag, err)) break;
-          } else if (!g_seen) {
-            if (!(g_seen = mbar_wait(&ms->g_full, 0, abort_flag, err))) break;
-          }
-          mbar_arrive_expect_tx(&ms->x_full[s], SB);
-          for (int jj = 0; jj < nblk; ++jj)
-            tma_load_3d(base + so + jj * 16384u, &tm_x, &ms->x_full[s], h * TP, t0 + 128 * jj, bi);
+        if (k >= NS) {
+          if (!mbar_wait(&ms->x_free[s], (u - 1) & 1, abort_flag, err)) break;
+        } else if (!g_seen) {
+          if (!(g_seen = mbar_wait(&ms->g_full, 0, abort_flag, err))) break;
         }
-        for (int kn = 0; kn < 2; ++kn)
-          tma_load_3d(base + so + (uint32_t)nblk * 16384u + kn * 8192u, &tm_h, &ms->x_full[s], 64 * kn, 0,
-                      (bi * nc + c) * d.H + h);
+        mbar_arrive_expect_tx(&ms->x_full[s], SBX);
+        tma_load_3d(base + so, xm, &ms->x_full[s], h * TP, t0, bi);
         issued = k + 1;
       }
       if (*abort_flag) {  // let this CTA's own loads land before it exits
@@ -677,7 +697,7 @@ k_chunk_scan_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
       bool prev_steep = false;
       for (int k = 0; ok && k < nh; ++k) {
         const int s = k % NS, u = k / NS, a = k & 1, cb = k % K3_CUMBUF;
-        if (!mbar_wait(&ms->x_full[s], u & 1, abort_flag, err)) break;
+        if (!mbar_wait(&ms->h_full[s], u & 1, abort_flag, err)) break;
         if (k >= 2 && !mbar_wait(&ms->acc_free[a], ((k >> 1) - 1) & 1, abort_flag, err)) break;
         // a steep head k-1 keeps its own W in this head's buffer until its MMAs are done
         if (prev_steep && !mbar_wait(&ms->x_free[(k - 1) % NS], ((k - 1) / NS) & 1, abort_flag, err)) break;
@@ -686,7 +706,7 @@ k_chunk_scan_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
         tc_fence_after();
         const uint32_t acc = tmem + k3_buf(a);
         const uint32_t so = smem_u32(base + K3Smem::slot(nblk, s));
-        const uint32_t hsa = so + (uint32_t)nblk * 16384u;
+        const uint32_t hsa = so + SBX;
         // ACC_inter = C_tile h_prev^T: K = d_state
         for (int ks = 0; ks < 8; ++ks) {
           const uint64_t ad = smem_desc_sw128(cm + (ks >> 2) * 16384u + (ks & 3) * 32u, 16u, 1024u);
@@ -696,6 +716,34 @@ k_chunk_scan_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
         mma_commit(&ms->acc_full[a]);
         mma_commit(&ms->x_free[s]);
       }
+    }
+    __syncwarp();
+  } else if (warp == 21) {
+    // ------------------------------------------------------------- TMA: entering states
+    // One box per head (both 64-wide halves of d_state, as the state-passing kernel stores
+    // them) into the slot after the head's x, on its own barrier.  The slot is reused once
+    // the three MMA issuers have released it; a slot overlapping the B rows only once G
+    // has been formed.
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_h);
+      const uint32_t bmo = K3Smem::bm(nblk);
+      grid_dep_wait();  // the entering states are the state-passing kernel's output
+      bool g_seen = false;
+      int issued = 0;
+      for (int k = 0; k < nh; ++k) {
+        const int s = k % NS, u = k / NS;
+        const uint32_t so = K3Smem::slot(nblk, s);
+        if (k >= NS) {
+          if (!mbar_wait(&ms->x_free[s], (u - 1) & 1, abort_flag, err)) break;
+        } else if (so + SB > bmo && !g_seen) {
+          if (!(g_seen = mbar_wait(&ms->g_full, 0, abort_flag, err))) break;
+        }
+        mbar_arrive_expect_tx(&ms->h_full[s], 16384u);
+        tma_load_3d(base + so + SBX, &tm_h, &ms->h_full[s], 0, 0, (bi * nc + c) * d.H + h0 + k);
+        issued = k + 1;
+      }
+      if (*abort_flag)  // let this CTA's own loads land before it exits
+        for (int k = (issued > NS ? issued - NS : 0); k < issued; ++k) mbar_wait_drain(&ms->h_full[k % NS], (k / NS) & 1);
     }
     __syncwarp();
   } else if (warp < 6 || warp >= 17) {
@@ -1030,22 +1078,82 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
+// Encoded tensor maps of recent calls.  A map depends only on its encoding arguments (the
+// address, the extents and the box), so a cached one is reused whenever all of them match;
+// the cache never dereferences the address.  Serving loops that call the prefill with the
+// same buffers every time then skip the host-side encoding.
+struct MapKey {
+  int type;
+  uint32_t esize, inner, rows;
+  const void *ptr;
+  uint64_t d0, d1, d2;
+  bool operator==(const MapKey &o) const {
+    return type == o.type && esize == o.esize && inner == o.inner && rows == o.rows && ptr == o.ptr && d0 == o.d0 &&
+           d1 == o.d1 && d2 == o.d2;
+  }
+};
+constexpr int kMapCacheSize = 64;
+struct MapCache {
+  std::mutex mu;
+  MapKey key[kMapCacheSize];
+  CUtensorMap map[kMapCacheSize];
+  int used = 0, next = 0;
+};
+MapCache &map_cache() {
+  static MapCache c;
+  return c;
+}
+
 // 3-D tensor map {d0 (contiguous), d1, d2}, box {inner, rows, 1}, 128-byte swizzle.
 bool make_map_t(CUtensorMap *m, CUtensorMapDataType type, uint32_t esize, const void *ptr, uint64_t d0, uint64_t d1,
                 uint64_t d2, uint32_t inner, uint32_t rows) {
+  const MapKey k{(int)type, esize, inner, rows, ptr, d0, d1, d2};
+  MapCache &c = map_cache();
+  {
+    std::lock_guard<std::mutex> lock(c.mu);
+    for (int i = 0; i < c.used; ++i)
+      if (c.key[i] == k) {
+        *m = c.map[i];
+        return true;
+      }
+  }
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   const cuuint64_t dims[3] = {d0, d1, d2};
   const cuuint64_t strides[2] = {d0 * esize, d0 * d1 * esize};
   const cuuint32_t box[3] = {inner, rows, 1};
   const cuuint32_t estr[3] = {1, 1, 1};
-  return fn(m, type, 3, const_cast<void *>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  if (fn(m, type, 3, const_cast<void *>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return false;
+  std::lock_guard<std::mutex> lock(c.mu);
+  const int slot = c.used < kMapCacheSize ? c.used++ : (c.next++ % kMapCacheSize);
+  c.key[slot] = k;
+  c.map[slot] = *m;
+  return true;
 }
 // 3-D bf16 tensor map {d0 (contiguous), d1, d2} with a {64, rows, 1} box and 128-byte swizzle.
 bool make_map(CUtensorMap *m, const void *ptr, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t rows) {
   return make_map_t(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ptr, d0, d1, d2, 64, rows);
+}
+
+size_t k1_smem_bytes(int Q) { return 1024 + K1Smem::misc(Q) + sizeof(K1Misc); }
+
+// The kernels' dynamic shared-memory limits, raised once per device (a per-function
+// attribute of the current device's module) to the largest size any call launches with:
+// chunk_state's for Q = 256, chunk_scan's fixed size.
+cudaError_t set_smem_limits_once() {
+  static std::atomic<uint64_t> done{0};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const uint64_t bit = dev < 64 ? (uint64_t)1 << dev : 0;
+  if (bit && (done.load(std::memory_order_acquire) & bit)) return cudaSuccess;
+  e = cudaFuncSetAttribute(k_chunk_state_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)k1_smem_bytes(256));
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(k_chunk_scan_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kK3SmemBytes);
+  if (e == cudaSuccess && bit) done.fetch_or(bit, std::memory_order_acq_rel);
+  return e;
 }
 
 int num_sms() {
@@ -1160,7 +1268,7 @@ cudaError_t launch_after(dim3 grid, unsigned threads, size_t smem, cudaStream_t 
 
 bool tc_prefill_supported(const Dims &d, int Q) { return d.P == TP && d.N == TN && (Q == 128 || Q == 256); }
 
-size_t tc_prefill_smem_k1(int Q) { return 1024 + K1Smem::misc(Q) + sizeof(K1Misc); }
+size_t tc_prefill_smem_k1(int Q) { return k1_smem_bytes(Q); }
 size_t tc_prefill_table_floats(const Dims &d, int Q, int nc) { return (size_t)d.b * d.H * nc * tab_row_floats(Q); }
 size_t tc_prefill_smem_k3() { return kK3SmemBytes; }
 
@@ -1168,12 +1276,13 @@ cudaError_t launch_tc_prefill(const __nv_bfloat16 *x, const float *dt, const flo
                               const __nv_bfloat16 *C, const float *D, const float *init, float *y, float *final_state,
                               float *cstates, float *tab, float *states, float *cdecay, __nv_bfloat16 *hprev, int *err,
                               const Dims &d, int Q, int nc, cudaStream_t st, const cudaEvent_t *ev) {
-  CUtensorMap tm_x1, tm_B1, tm_x3, tm_C3, tm_B3, tm_h3, tm_y3;
+  CUtensorMap tm_x1, tm_B1, tm_x3, tm_x3b, tm_C3, tm_B3, tm_h3, tm_y3;
   const uint64_t HP = (uint64_t)d.H * d.P, GN = (uint64_t)d.G * d.N;
   if (!make_map(&tm_x1, x, HP, d.L, d.b, Q) || !make_map(&tm_B1, B, GN, d.L, d.b, Q) ||
-      !make_map(&tm_x3, x, HP, d.L, d.b, 128) || !make_map(&tm_C3, C, GN, d.L, d.b, 128) ||
+      !make_map(&tm_x3, x, HP, d.L, d.b, 128) || !make_map(&tm_x3b, x, HP, d.L, d.b, 256) ||
+      !make_map(&tm_C3, C, GN, d.L, d.b, 128) ||
       !make_map(&tm_B3, B, GN, d.L, d.b, 128) ||
-      !make_map(&tm_h3, hprev, (uint64_t)d.N, (uint64_t)d.P, (uint64_t)d.b * nc * d.H, 64) ||
+      !make_map(&tm_h3, hprev, 64, 2 * (uint64_t)d.P, (uint64_t)d.b * nc * d.H, 2 * d.P) ||
       !make_map_t(&tm_y3, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, y, HP, d.L, d.b, 32, 32))
     return cudaErrorInvalidValue;
   const int sms = num_sms();
@@ -1183,24 +1292,25 @@ cudaError_t launch_tc_prefill(const __nv_bfloat16 *x, const float *dt, const flo
   const bool pdl = ev == nullptr;
   cudaError_t e = mark(0);
   if (e != cudaSuccess) return e;
+  if ((e = set_smem_limits_once()) != cudaSuccess) return e;
   // K1
   {
     const int base_items = d.b * nc * d.G;
     const int kb = std::min(K1_KB_MAX, pick_heads_per_cta(base_items, d.hpg, sms, 1.0));
     const int nhb = (d.hpg + kb - 1) / kb;
-    const size_t smem = tc_prefill_smem_k1(Q);
-    e = cudaFuncSetAttribute(k_chunk_state_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    e = launch_after(dim3((unsigned)(base_items * nhb)), K1_THREADS, tc_prefill_smem_k1(Q), st, pdl, k_chunk_state_tc,
+                     tm_x1, tm_B1, dt, A, D, tab, cdecay, states, err, d, Q, nc, kb, nhb);
     if (e != cudaSuccess) return e;
-    k_chunk_state_tc<<<(unsigned)(base_items * nhb), K1_THREADS, smem, st>>>(tm_x1, tm_B1, dt, A, D, tab, cdecay,
-                                                                             states, err, d, Q, nc, kb, nhb);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   if ((e = mark(1)) != cudaSuccess) return e;
   // K2
   {
     const int per_head = d.P * d.N / 4;
-    e = launch_after(dim3(d.b * d.H, (per_head + K2_THREADS - 1) / K2_THREADS), K2_THREADS, kK2SmemBytes, st, pdl,
-                     k_state_passing_bf16, states, cdecay, hprev, init, final_state, cstates, d, nc);
+    const dim3 grid(d.b * d.H, (per_head + K2_THREADS - 1) / K2_THREADS);
+    e = cstates ? launch_after(grid, K2_THREADS, kK2SmemBytes, st, pdl, k_state_passing_bf16<true>, states, cdecay,
+                               hprev, init, final_state, cstates, d, nc)
+                : launch_after(grid, K2_THREADS, kK2SmemBytes, st, pdl, k_state_passing_bf16<false>, states, cdecay,
+                               hprev, init, final_state, cstates, d, nc);
     if (e != cudaSuccess) return e;
   }
   if ((e = mark(2)) != cudaSuccess) return e;
@@ -1209,10 +1319,8 @@ cudaError_t launch_tc_prefill(const __nv_bfloat16 *x, const float *dt, const flo
     const int ntt = Q / 128;
     const int groups = d.b * nc * d.G;
     const ScanSplit sp = pick_scan_split(groups, d.hpg, ntt, sms);
-    e = cudaFuncSetAttribute(k_chunk_scan_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kK3SmemBytes);
-    if (e != cudaSuccess) return e;
     e = launch_after(dim3((unsigned)(groups * (sp.nhb0 + sp.nhb1))), K3_THREADS, kK3SmemBytes, st, pdl,
-                     k_chunk_scan_tc, tm_x3, tm_C3, tm_B3, tm_h3, tm_y3, (const float *)tab, err, d, Q, nc, sp.kb0,
+                     k_chunk_scan_tc, tm_x3, tm_x3b, tm_C3, tm_B3, tm_h3, tm_y3, (const float *)tab, err, d, Q, nc, sp.kb0,
                      sp.nhb0, sp.kb1, sp.nhb1);
     if (e != cudaSuccess) return e;
   }

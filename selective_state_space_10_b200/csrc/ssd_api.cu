@@ -198,8 +198,8 @@ static ssd_status prefill_impl(const ssd_dims *dims, ssd_dtype dtype, const void
   }
   char *ws = static_cast<char *>(workspace);
   cudaEvent_t const *ev = timed ? reinterpret_cast<cudaEvent_t const *>(events) : nullptr;
-  cudaError_t e = cudaMemsetAsync(ws, 0, sizeof(int), st);  // device error word
-  if (e != cudaSuccess) return SSD_ERR_CUDA;
+  // The device error word starts at zero: the tensor-core path's first kernel clears it
+  // itself; the CUDA-core path (which has no bounded waits) clears it here.
   if (pl.path == Path::kTensorCore)
     return cuda_status(ssd::launch_tc_prefill(
         static_cast<const __nv_bfloat16 *>(x), dt, A, static_cast<const __nv_bfloat16 *>(B),
@@ -207,6 +207,7 @@ static ssd_status prefill_impl(const ssd_dims *dims, ssd_dtype dtype, const void
         reinterpret_cast<float *>(ws + pl.states_off),
         reinterpret_cast<float *>(ws + pl.cdecay_off), reinterpret_cast<__nv_bfloat16 *>(ws + pl.hprev_off),
         reinterpret_cast<int *>(ws), d, chunk, pl.nc, st, ev));
+  if (cudaMemsetAsync(ws, 0, sizeof(int), st) != cudaSuccess) return SSD_ERR_CUDA;
   if (dtype == SSD_F32)
     return run_prefill<float>(d, chunk, pl, static_cast<const float *>(x), dt, A, static_cast<const float *>(B),
                               static_cast<const float *>(C), D, init, y, final_state, cstates, ws, st, ev);

@@ -34,8 +34,9 @@ class Dims(ctypes.Structure):
 EXPORTS = ("ssd_status_string", "ssd_version", "ssd_prefill_workspace_size",
            "ssd_prefill_kernel_launches", "ssd_prefill", "ssd_prefill_ex", "ssd_prefill_timed",
            "ssd_prefill_kernel_name", "ssd_prefill_device_status", "ssd_prefill_noalloc",
-           "ssd_prefill_noalloc_max_workspace", "ssd_decode_step", "ssd_frontend", "ssd_decode_window_step",
-           "ssd_decode_window_flush", "ssd_wait_selftest", "ssd_prefill_host_buffer_size", "ssd_prefill_host")
+           "ssd_prefill_noalloc_max_workspace", "ssd_prefill_noalloc_device_status", "ssd_decode_step",
+           "ssd_frontend", "ssd_decode_window_step", "ssd_decode_window_flush", "ssd_wait_selftest",
+           "ssd_prefill_host_buffer_size", "ssd_prefill_host")
 
 
 def _load():
@@ -68,6 +69,8 @@ def _load():
     lib.ssd_prefill_noalloc.restype = ci
     lib.ssd_prefill_noalloc_max_workspace.argtypes = []
     lib.ssd_prefill_noalloc_max_workspace.restype = sz
+    lib.ssd_prefill_noalloc_device_status.argtypes = [vp]
+    lib.ssd_prefill_noalloc_device_status.restype = ci
     lib.ssd_prefill_host_buffer_size.argtypes = [dp, ci, ci]
     lib.ssd_prefill_host_buffer_size.restype = sz
     lib.ssd_prefill_host.argtypes = [dp, ci, vp, fp, fp, vp, vp, fp, ci, fp, fp, vp, sz, vp]
@@ -289,6 +292,12 @@ def prefill_noalloc(x, dt, A, B, C, D, chunk: int = 256, y=None, final_state=Non
 
 def prefill_noalloc_max_workspace() -> int:
     return lib.ssd_prefill_noalloc_max_workspace()
+
+
+def prefill_noalloc_device_status(stream=None) -> int:
+    """ssd_prefill_noalloc_device_status: waits for the stream and returns OK or
+    ERR_TIMEOUT from the error word of the library's scratch array."""
+    return lib.ssd_prefill_noalloc_device_status(_stream(stream))
 
 
 def prefill_device_status(workspace, stream=None) -> int:

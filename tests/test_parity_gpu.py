@@ -178,7 +178,7 @@ def test_full_prefill_workloads(ssd, name):
 def test_long_context_prefill_then_decode(ssd):
     """b=4, L=16384 prefill, then 256 decode steps from its final state, against (i) one
     GPU prefill of all 16640 tokens (every head) and (ii) the oracle over all 16640
-    tokens on a sample of (batch row, head) pairs."""
+    tokens, every (batch row, head) pair: y of every token and the final state."""
     w = inputs.BY_NAME["mamba2_130m_long_b4"]
     full = inputs.workload_sequence(w, seqlen=w.seqlen + w.decode_steps)
     pre = full.token_slice(0, w.seqlen)
@@ -196,29 +196,44 @@ def test_long_context_prefill_then_decode(ssd):
     y_split, y_one = y_split.cpu().numpy(), y_one.cpu().numpy()
     assert_close(y_split, y_one, 2e-2, "split vs one prefill y")
     assert_close(state.cpu().numpy(), fs_one.cpu().numpy(), 2e-2, "split vs one prefill state")
-    rng = np.random.default_rng(0)
-    for bi, h in [(0, 0), (3, 23)] + [tuple(v) for v in rng.integers((0, 0), (4, 24), (2, 2))]:
-        hs = full.head_slice(bi, h)
-        y_ref, fs_ref = oracle.recurrence(hs.x, hs.dt, hs.A, hs.B, hs.C, hs.D)
-        assert_close(y_split[bi:bi + 1, :, h:h + 1], y_ref, 2e-2, f"oracle y (b={bi}, h={h})")
-        assert_close(state.cpu().numpy()[bi:bi + 1, h:h + 1], fs_ref, 2e-2, f"oracle state (b={bi}, h={h})")
+    y_ref, fs_ref = oracle.recurrence(full.x, full.dt, full.A, full.B, full.C, full.D)
+    st = state.cpu().numpy()
+    assert_close(y_split, y_ref, 2e-2, "oracle y, all 96 (batch row, head) pairs")
+    assert_close(st, fs_ref, 2e-2, "oracle final state, all 96 pairs")
+    for bi in range(w.batch):  # and each pair on its own scale, so that no small head hides
+        for h in range(w.nheads):
+            assert_close(y_split[bi, :, h], y_ref[bi, :, h], 2e-2, f"oracle y (b={bi}, h={h})")
+            assert_close(st[bi, h], fs_ref[bi, h], 2e-2, f"oracle state (b={bi}, h={h})")
 
 
 def test_batched_decode_workload(ssd):
-    """batch 256 x 80 heads, 1024 decode steps from a seeded N(0, 0.1^2) state; y checked
-    against the oracle at steps 0..15, 31, 63, ..., 1023 and the final state, on a sample
-    of (batch row, head) pairs (the oracle runs only those)."""
+    """batch 256 x 80 heads, 1024 decode steps from a seeded N(0, 0.1^2) state.  Every one
+    of the 20480 heads is checked against the oracle (y and the whole state) after step 0
+    and after step 15, the oracle stepping all heads; then y at steps 31, 63, ..., 1023
+    and the final state on a sample of (batch row, head) pairs, the oracle continuing
+    only those."""
     w = inputs.BY_NAME["mamba2_2.7b_decode_b256"]
     state0 = inputs.decode_initial_state(w)
     state = torch.from_numpy(state0).cuda()
     rng = np.random.default_rng(1)
     pairs = [(0, 0), (255, 79)] + [tuple(v) for v in rng.integers((0, 0), (256, 80), (10, 2))]
-    st_ref = {p: state0[p[0]:p[0] + 1, p[1]:p[1] + 1].astype(np.float64) for p in pairs}
+    full_steps = 16
+    st_all = state0.astype(np.float64)
     checks = set(range(16)) | {31, 63, 127, 255, 511, 1023}
     worst = 0.0
+    st_ref = {}
     for step in range(w.decode_steps):
         tok = inputs.decode_token(w, step)
         y = ssd.decode_step(state, **decode_args(to_device(tok)))
+        if step < full_steps:  # the oracle steps every head
+            y_ref, st_all = oracle.recurrence(tok.x, tok.dt, tok.A, tok.B, tok.C, tok.D, state=st_all)
+            if step in (0, full_steps - 1):
+                worst = max(worst, assert_close(y.cpu().numpy(), y_ref[:, 0], 2e-2, f"step {step}: y, all heads"))
+                assert_close(state.cpu().numpy(), st_all, 2e-2, f"step {step}: state, all heads")
+            if step == full_steps - 1:
+                st_ref = {p: st_all[p[0]:p[0] + 1, p[1]:p[1] + 1].copy() for p in pairs}
+                del st_all
+            continue
         for (bi, h) in pairs:
             hs = tok.head_slice(bi, h)
             y_ref, st_ref[(bi, h)] = oracle.recurrence(hs.x, hs.dt, hs.A, hs.B, hs.C, hs.D,

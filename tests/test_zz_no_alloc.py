@@ -48,6 +48,8 @@ def test_noalloc_matches_prefill_on_consecutive_calls(ssd):
         assert_close(y, y_ref, TOL[dtype], f"call {i}: y")
         assert_close(fs, fs_ref, TOL[dtype], f"call {i}: final state")
         assert np.array_equal(y, y_ref) and np.array_equal(fs, fs_ref), "same kernels: results should be identical"
+        # the caller holds no workspace: the scratch array's own error word reports the waits
+        assert ssd.prefill_noalloc_device_status() == ssd.OK
 
 
 def test_noalloc_rejects_problems_larger_than_its_scratch(ssd):
