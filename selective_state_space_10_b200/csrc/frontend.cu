@@ -109,9 +109,10 @@ k_frontend(const T *__restrict__ xbc, const float *__restrict__ w, const float *
   const int t1 = min(t0 + kFeTokens, d.L);
   // Stage this CTA's inputs -- rows t0-3 .. t1-1 of its 256 * V channels -- in shared
   // memory with asynchronous copies (nothing held in registers while they fly): with 4
-  // channels a thread, one bulk copy per row by one thread, completing on an mbarrier;
-  // otherwise a cp.async per thread and row.  Rows before the sequence come from the conv
-  // state or are zero.
+  // channels a thread, one bulk copy per row, the rows spread over the eight warps (a
+  // thread completes about one bulk copy per half microsecond), each warp arriving on the
+  // mbarrier with its own byte count; otherwise a cp.async per thread and row.  Rows before
+  // the sequence come from the conv state or are zero.
   __shared__ __align__(16) T tile[3 + kFeTokens][256 * V];
   __shared__ uint64_t rows_full;
   const int tl = threadIdx.x * V;  // this thread's first channel within the tile
@@ -120,24 +121,27 @@ k_frontend(const T *__restrict__ xbc, const float *__restrict__ w, const float *
   const bool bulk = V == 4 && (nch * (int)sizeof(T)) % 16 == 0 && ((size_t)CH * sizeof(T)) % 16 == 0 &&
                     reinterpret_cast<uintptr_t>(xbc) % 16 == 0;
   const T *uc = xbc + (size_t)bi * d.L * CH + c;
+  const int nwarps = blockDim.x >> 5, warp = threadIdx.x >> 5;
   if (bulk) {
     if (threadIdx.x == 0) {
-      sm100::mbar_init(&rows_full, 1);
+      sm100::mbar_init(&rows_full, nwarps);
       sm100::mbar_fence_init();
+    }
+    __syncthreads();  // the barrier is initialised before any thread arrives on it
+    if ((threadIdx.x & 31) == 0) {
       uint32_t bytes = 0;
-      for (int j = 0; j < 3 + kFeTokens; ++j) {
+      for (int j = warp; j < 3 + kFeTokens; j += nwarps) {
         const int t = t0 - 3 + j;
         if (t >= 0 && t < t1) bytes += (uint32_t)nch * sizeof(T);
       }
       sm100::mbar_arrive_expect_tx(&rows_full, bytes);
-      for (int j = 0; j < 3 + kFeTokens; ++j) {
+      for (int j = warp; j < 3 + kFeTokens; j += nwarps) {
         const int t = t0 - 3 + j;
         if (t >= 0 && t < t1)
           sm100::bulk_load(&tile[j][0], xbc + ((size_t)bi * d.L + t) * CH + cbase, (uint32_t)nch * sizeof(T),
                            &rows_full);
       }
     }
-    __syncthreads();  // the barrier is initialised before any thread waits on it
   } else if (active) {
 #pragma unroll
     for (int j = 0; j < 3 + kFeTokens; ++j) {
@@ -246,19 +250,25 @@ k_frontend_stream(const T *__restrict__ xbc, const float *__restrict__ w, const 
   const bool active = c < CH;
   const int nruns = (T1 - T0 + R - 1) / R;
   const T *rows = xbc + (size_t)bi * d.L * CH + cbase;  // row t of this tile at rows + t * CH
-  // run i into buffer i % kFeBufs: one bulk copy per row, by thread 0
+  // run i into buffer i % kFeBufs: one bulk copy per row, the rows spread over the eight
+  // warps (lane 0 of each), each arriving on the buffer's barrier with its own byte count
+  const int nwarps = blockDim.x >> 5, warp = threadIdx.x >> 5;
   auto issue = [&](int i) {
     const int ta = T0 + i * R, nr = min(R, T1 - ta);
     uint64_t *bar = &full[i % kFeBufs];
-    sm100::mbar_arrive_expect_tx(bar, (uint32_t)(nr * nch * (int)sizeof(T)));
-    for (int j = 0; j < nr; ++j)
+    uint32_t bytes = 0;
+    for (int j = warp; j < nr; j += nwarps) bytes += (uint32_t)nch * sizeof(T);
+    sm100::mbar_arrive_expect_tx(bar, bytes);
+    for (int j = warp; j < nr; j += nwarps)
       sm100::bulk_load(&buf[i % kFeBufs][j][0], rows + (size_t)(ta + j) * CH, (uint32_t)nch * sizeof(T), bar);
   };
   if (threadIdx.x == 0) {
-    for (int b = 0; b < kFeBufs; ++b) sm100::mbar_init(&full[b], 1);
+    for (int b = 0; b < kFeBufs; ++b) sm100::mbar_init(&full[b], nwarps);
     sm100::mbar_fence_init();
-    for (int i = 0; i < kFeBufs && i < nruns; ++i) issue(i);
   }
+  __syncthreads();  // the barriers are initialised before any warp arrives on them
+  if ((threadIdx.x & 31) == 0)
+    for (int i = 0; i < kFeBufs && i < nruns; ++i) issue(i);
   {  // dt for this range of tokens and this tile's share of the heads
     const int per = (d.H + gridDim.y - 1) / gridDim.y, hlo = blockIdx.y * per, nhs = min(per, d.H - hlo);
     const int count = nhs > 0 ? (T1 - T0) * nhs : 0;
@@ -302,7 +312,6 @@ k_frontend_stream(const T *__restrict__ xbc, const float *__restrict__ w, const 
     dst = C + (size_t)bi * d.L * GN + (c - HP - GN);
     stride = GN;
   }
-  __syncthreads();  // the barriers are initialised before any thread waits on them
   bool ok = true;
   int waited = 0;  // runs whose copies this thread has seen land
   for (int i = 0; i < nruns; ++i) {
@@ -328,7 +337,7 @@ k_frontend_stream(const T *__restrict__ xbc, const float *__restrict__ w, const 
       }
     }
     __syncthreads();  // every thread has read buffer i % kFeBufs
-    if (threadIdx.x == 0 && ok && i + kFeBufs < nruns) issue(i + kFeBufs);
+    if ((threadIdx.x & 31) == 0 && ok && i + kFeBufs < nruns) issue(i + kFeBufs);
   }
   if (!ok && threadIdx.x == 0) {  // let this CTA's own copies land before it exits
     const int issued = min(nruns, waited + kFeBufs);

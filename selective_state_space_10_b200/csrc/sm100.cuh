@@ -84,12 +84,13 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
   }
 }
 
-// Bounded wait that ignores the abort flag: used at teardown to let this CTA's own
-// copies in flight land before it exits.  Returns false if the limit expired.
+// Bounded wait that ignores the abort flag (sleeping on the barrier between checks, as
+// mbar_wait): used at teardown to let this CTA's own copies in flight land before it
+// exits, and by kernels without an abort flag.  Returns false if the limit expired.
 __device__ __forceinline__ bool mbar_wait_drain(uint64_t *bar, uint32_t parity, uint64_t limit_ns = 1000000000ull) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
-  while (!mbar_try_wait(bar, parity))
+  while (!mbar_try_wait_sleep(bar, parity, 20000u))
     if (globaltimer_ns() - t0 > limit_ns) return false;
   return true;
 }
