@@ -375,7 +375,139 @@ k_chunk_state_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
 }
 
 // ============================================================================ K2
-// grid (b * H, ceil(P*N/4 / 256)), block 256: one float4 of the state per thread.  The
+// State passing: h_c = exp(cum_end,c) h_{c-1} + S_c over the chunks, in fp32 (the
+// first-order recurrence of "Mamba and Selective State Space Models" section 5), for every
+// float4 column of every (batch, head) state.  Two kernels: for sequences of more than
+// K2_ROUND chunks (measured faster there), one wave of CTAs, one per SM: each owns a
+// contiguous range of a batch row's state columns (heads x P x N / 4), which for a given
+// chunk is one contiguous span of the chunk states.  The spans of several chunks at a time
+// are staged in shared memory by bulk copies (one per chunk, issued from different warps,
+// since a thread completes about one copy per half microsecond) into two buffers, so the
+// next chunks fly while one buffer is read; each thread keeps the running state of its
+// columns in registers.
+//
+// The chunk states S (fp32) and the bf16 entering states of a (batch, chunk, head) share
+// one layout, the two 64-wide halves of d_state, [n / 64][p][n % 64] (d_state = 128), so
+// that the chunk-scan kernel fetches an entering state with one box; a column index e4
+// addresses four consecutive elements of that layout, and the same four elements of a
+// [p][n] state (initial, final, exported chunk states) are at state_column_pn(e4).  The
+// recurrence starts from `init` (zero if NULL; it may alias final_state: every CTA reads
+// the initial values of its columns before it writes any final value); with `cstates`
+// non-NULL the state after every chunk is also written there.
+constexpr int K2_THREADS = 512;
+constexpr int K2_MAX_COLS = 4;                 // columns a thread owns at most
+constexpr size_t kK2Buf = 104u * 1024u;        // bytes of a staging buffer
+constexpr size_t kK2SmemBytes = 2 * kK2Buf;
+
+__device__ __forceinline__ int state_column_pn(int e4, const Dims &d) {
+  const int half = (4 * e4) / (d.P * 64), rem = 4 * e4 - half * d.P * 64;
+  return ((rem >> 6) * d.N + half * 64 + (rem & 63)) >> 2;
+}
+
+__global__ void __launch_bounds__(K2_THREADS, 1)
+k_state_passing_bf16(const float *__restrict__ states, const float *__restrict__ cdecay,
+                     __nv_bfloat16 *__restrict__ hprev, const float *init, float *final_state,
+                     float *__restrict__ cstates, int *err, Dims d, int nc, int cpc, int parts) {
+  extern __shared__ __align__(16) uint8_t k2_smem[];
+  __shared__ uint64_t full[2];
+  const int PN4 = d.P * d.N / 4;
+  const int rowcols = d.H * PN4;  // state columns of one batch row
+  const int bi = blockIdx.x / parts, part = blockIdx.x % parts;
+  const int col0 = part * cpc, ncol = min(cpc, rowcols - col0);
+  const int nwarps = K2_THREADS / 32, warp = threadIdx.x >> 5;
+  sm100::grid_dep_launch();  // the chunk scan may start its own set-up meanwhile
+  if (ncol <= 0) return;
+  const int ks = max(1, min(nc, (int)(kK2Buf / ((size_t)ncol * sizeof(float4)))));  // chunks per stage
+  const int nstage = (nc + ks - 1) / ks;
+  const size_t cstride = (size_t)rowcols;  // float4s between consecutive chunks
+  const float4 *src = reinterpret_cast<const float4 *>(states) + (size_t)bi * nc * cstride + col0;
+  float4 *buf0 = reinterpret_cast<float4 *>(k2_smem);
+  float4 *buf1 = reinterpret_cast<float4 *>(k2_smem + kK2Buf);
+  if (threadIdx.x == 0) {
+    sm100::mbar_init(&full[0], nwarps);
+    sm100::mbar_init(&full[1], nwarps);
+    sm100::mbar_fence_init();
+  }
+  __syncthreads();
+  sm100::grid_dep_wait();  // chunk states and decays of the chunk-state kernel
+  // stage st: chunk j of it by lane 0 of warp j % nwarps; every warp arrives with its bytes
+  auto issue = [&](int st) {
+    float4 *b = (st & 1) ? buf1 : buf0;
+    const int c0 = st * ks, cn = min(ks, nc - c0);
+    uint32_t bytes = 0;
+    for (int j = warp; j < cn; j += nwarps) bytes += (uint32_t)ncol * sizeof(float4);
+    sm100::mbar_arrive_expect_tx(&full[st & 1], bytes);
+    for (int j = warp; j < cn; j += nwarps)
+      sm100::bulk_load(b + (size_t)j * ncol, src + (size_t)(c0 + j) * cstride, (uint32_t)ncol * sizeof(float4),
+                       &full[st & 1]);
+  };
+  if ((threadIdx.x & 31) == 0)
+    for (int st = 0; st < 2 && st < nstage; ++st) issue(st);
+  // this thread's columns and their running states
+  float4 hs[K2_MAX_COLS];
+  const float *decp[K2_MAX_COLS];
+#pragma unroll
+  for (int i = 0; i < K2_MAX_COLS; ++i) {
+    const int cl = threadIdx.x + i * K2_THREADS;
+    hs[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    decp[i] = cdecay;
+    if (cl < ncol) {
+      const int col = col0 + cl, h = col / PN4, e4 = col - h * PN4;
+      decp[i] = cdecay + ((size_t)bi * d.H + h) * nc;
+      if (init) hs[i] = reinterpret_cast<const float4 *>(init)[((size_t)bi * d.H + h) * PN4 + state_column_pn(e4, d)];
+    }
+  }
+  uint2 *hp = reinterpret_cast<uint2 *>(hprev) + (size_t)bi * nc * cstride + col0;
+  bool ok = true;
+  for (int st = 0; st < nstage; ++st) {
+    // bounded wait (1 s): on expiry the error word is raised and the outputs are undefined
+    ok = ok && sm100::mbar_wait_drain(&full[st & 1], (uint32_t)((st >> 1) & 1));
+    if (!ok && threadIdx.x == 0) atomicExch(err, 1);
+    const float4 *b = (st & 1) ? buf1 : buf0;
+    const int c0 = st * ks, cn = min(ks, nc - c0);
+    if (ok) {
+      for (int j = 0; j < cn; ++j) {
+        const int c = c0 + j;
+#pragma unroll
+        for (int i = 0; i < K2_MAX_COLS; ++i) {
+          const int cl = threadIdx.x + i * K2_THREADS;
+          if (cl < ncol) {
+            const float4 sv = b[(size_t)j * ncol + cl];
+            const float dc = __ldg(decp[i] + c);
+            hp[(size_t)c * cstride + cl] = make_uint2(sm100::pack_bf16x2(hs[i].x, hs[i].y),
+                                                      sm100::pack_bf16x2(hs[i].z, hs[i].w));
+            hs[i].x = fmaf(dc, hs[i].x, sv.x);
+            hs[i].y = fmaf(dc, hs[i].y, sv.y);
+            hs[i].z = fmaf(dc, hs[i].z, sv.z);
+            hs[i].w = fmaf(dc, hs[i].w, sv.w);
+            if (cstates) {  // state after chunk c, in the [p][n] layout
+              const int col = col0 + cl, h = col / PN4, e4 = col - h * PN4;
+              reinterpret_cast<float4 *>(cstates)[(((size_t)bi * nc + c) * d.H + h) * PN4 + state_column_pn(e4, d)] = hs[i];
+            }
+          }
+        }
+      }
+    }
+    __syncthreads();  // every thread has read this buffer
+    if ((threadIdx.x & 31) == 0 && ok && st + 2 < nstage) issue(st + 2);
+  }
+  if (!ok) {  // let this CTA's own copies land before it exits
+    if (threadIdx.x == 0)
+      for (int st = 0; st < 2 && st < nstage; ++st) sm100::mbar_wait_drain(&full[st & 1], 0);
+    return;
+  }
+#pragma unroll
+  for (int i = 0; i < K2_MAX_COLS; ++i) {
+    const int cl = threadIdx.x + i * K2_THREADS;
+    if (cl < ncol) {
+      const int col = col0 + cl, h = col / PN4, e4 = col - h * PN4;
+      reinterpret_cast<float4 *>(final_state)[((size_t)bi * d.H + h) * PN4 + state_column_pn(e4, d)] = hs[i];
+    }
+  }
+}
+
+// Short sequences (at most K2_ROUND chunks): grid (b * H, ceil(P*N/4 / 256)), block 256,
+// one float4 column of the state per thread, all of its chunks fetched at once.  The
 // update is sequential over chunks, so the time goes in waiting for the chunk states: a
 // thread fetches K2_ROUND chunks at once, half into registers and half into shared memory
 // by cp.async (which holds no register), so that a CTA has a whole round in flight after
@@ -383,11 +515,11 @@ k_chunk_state_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
 // stored in bf16, the final state in fp32.  The recurrence starts from `init` (zero if
 // NULL); with `cstates` non-NULL the state after every chunk is also written there in
 // fp32.  `init` may be final_state: each thread reads its element before it writes it.
-constexpr int K2_THREADS = 256;
+constexpr int K2R_THREADS = 256;
 constexpr int K2_REG = 8;              // chunks of a round held in registers
 constexpr int K2_STAGED = 8;           // chunks of a round staged in shared memory
 constexpr int K2_ROUND = K2_REG + K2_STAGED;
-constexpr size_t kK2SmemBytes = (size_t)K2_STAGED * K2_THREADS * sizeof(float4);
+constexpr size_t kK2RSmemBytes = (size_t)K2_STAGED * K2R_THREADS * sizeof(float4);
 
 __device__ __forceinline__ void cp_async16(void *dst, const void *src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
@@ -396,11 +528,11 @@ __device__ __forceinline__ void cp_async16(void *dst, const void *src) {
 // kExport: also store the state after every chunk (cstates non-NULL); a separate
 // instantiation, so that the plain prefill's kernel holds no pointer for it.
 template <bool kExport>
-__global__ void __launch_bounds__(K2_THREADS, 4)
-k_state_passing_bf16(const float *__restrict__ states, const float *__restrict__ cdecay,
+__global__ void __launch_bounds__(K2R_THREADS, 4)
+k_state_passing_rounds(const float *__restrict__ states, const float *__restrict__ cdecay,
                      __nv_bfloat16 *__restrict__ hprev, const float *init, float *final_state,
                      float *__restrict__ cstates, Dims d, int nc) {
-  extern __shared__ float4 k2_stage[];  // [K2_STAGED][K2_THREADS]
+  extern __shared__ float4 k2_stage[];  // [K2_STAGED][K2R_THREADS]
   const int PN4 = d.P * d.N / 4;
   const int e4 = blockIdx.y * blockDim.x + threadIdx.x;
   sm100::grid_dep_launch();  // the chunk scan may start its own set-up meanwhile
@@ -435,7 +567,7 @@ k_state_passing_bf16(const float *__restrict__ states, const float *__restrict__
     // issue the whole round: chunks c0 .. c0+7 into registers, c0+8 .. c0+15 into shared memory
 #pragma unroll
     for (int j = 0; j < K2_STAGED; ++j)
-      if (c0 + K2_REG + j < nc) cp_async16(stage + j * K2_THREADS, sp + (size_t)(c0 + K2_REG + j) * cstride);
+      if (c0 + K2_REG + j < nc) cp_async16(stage + j * K2R_THREADS, sp + (size_t)(c0 + K2_REG + j) * cstride);
     asm volatile("cp.async.commit_group;" ::: "memory");
     float4 sv[K2_REG];
 #pragma unroll
@@ -447,7 +579,7 @@ k_state_passing_bf16(const float *__restrict__ states, const float *__restrict__
     asm volatile("cp.async.wait_group 0;" ::: "memory");  // this thread's own copies
 #pragma unroll
     for (int j = 0; j < K2_STAGED; ++j)
-      if (c0 + K2_REG + j < nc) step(c0 + K2_REG + j, stage[j * K2_THREADS]);
+      if (c0 + K2_REG + j < nc) step(c0 + K2_REG + j, stage[j * K2R_THREADS]);
   }
   reinterpret_cast<float4 *>(final_state)[own4] = hs;
 }
@@ -1152,6 +1284,8 @@ cudaError_t set_smem_limits_once() {
   e = cudaFuncSetAttribute(k_chunk_state_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)k1_smem_bytes(256));
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(k_chunk_scan_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kK3SmemBytes);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(k_state_passing_bf16, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kK2SmemBytes);
   if (e == cudaSuccess && bit) done.fetch_or(bit, std::memory_order_acq_rel);
   return e;
 }
@@ -1305,12 +1439,23 @@ cudaError_t launch_tc_prefill(const __nv_bfloat16 *x, const float *dt, const flo
   if ((e = mark(1)) != cudaSuccess) return e;
   // K2
   {
-    const int per_head = d.P * d.N / 4;
-    const dim3 grid(d.b * d.H, (per_head + K2_THREADS - 1) / K2_THREADS);
-    e = cstates ? launch_after(grid, K2_THREADS, kK2SmemBytes, st, pdl, k_state_passing_bf16<true>, states, cdecay,
-                               hprev, init, final_state, cstates, d, nc)
-                : launch_after(grid, K2_THREADS, kK2SmemBytes, st, pdl, k_state_passing_bf16<false>, states, cdecay,
-                               hprev, init, final_state, cstates, d, nc);
+    if (nc <= K2_ROUND) {  // every chunk of a column fetched at once by its thread
+      const int per_head = d.P * d.N / 4;
+      const dim3 grid(d.b * d.H, (per_head + K2R_THREADS - 1) / K2R_THREADS);
+      e = cstates ? launch_after(grid, K2R_THREADS, kK2RSmemBytes, st, pdl, k_state_passing_rounds<true>, states,
+                                 cdecay, hprev, init, final_state, cstates, d, nc)
+                  : launch_after(grid, K2R_THREADS, kK2RSmemBytes, st, pdl, k_state_passing_rounds<false>, states,
+                                 cdecay, hprev, init, final_state, cstates, d, nc);
+    } else {
+      // one wave: the batch rows' state columns split evenly over the SMs, at most
+      // K2_MAX_COLS per thread (more CTAs, in several waves, past that)
+      const long rowcols = (long)d.H * d.P * d.N / 4;
+      const long per_sm = ((long)d.b * rowcols + sms - 1) / sms;
+      const int cpc = (int)std::min<long>((long)K2_MAX_COLS * K2_THREADS, std::max<long>(per_sm, 1));
+      const int parts = (int)((rowcols + cpc - 1) / cpc);
+      e = launch_after(dim3((unsigned)(d.b * parts)), K2_THREADS, kK2SmemBytes, st, pdl, k_state_passing_bf16, states,
+                       cdecay, hprev, init, final_state, cstates, err, d, nc, cpc, parts);
+    }
     if (e != cudaSuccess) return e;
   }
   if ((e = mark(2)) != cudaSuccess) return e;
