@@ -973,25 +973,59 @@ k_chunk_scan_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
         }
       }
       // Each thread takes row tl of every x block of the slot (the 128-byte swizzle keeps 8
-      // consecutive rows on distinct banks).  In the tile's own block it first stores
-      // D x_t / u_t into the intra accumulator (the MMA adds W X' onto it); then, unless the
-      // head is steep (its W holds the decay), it scales the row by v_s in place.
+      // consecutive rows on distinct banks) and, unless the head is steep (its W holds the
+      // decay), scales it by v_s in place as soon as x has landed, keeping the raw values of
+      // the tile's own block.  Only then does it wait for the head's accumulator buffer and
+      // store D x_t / u_t into the intra accumulator (the MMA adds W X' onto it), so that the
+      // scaling is not part of the loop "buffer released -> MMAs -> read out -> released".
       ok = ok && mbar_wait(&ms->x_full[s], (k / NS) & 1, abort_flag, err);
+      // A split head's rows and sources from m = 128*ti + 64 on take the second reference,
+      // and their D x_t / u_t goes to the second intra accumulator (the first gets 0 for
+      // them, and the second gets 0 for the rows before m).
+      const bool second = td.split && tl >= 64;
+      uint32_t own[16];  // raw x of row tl, channels 32 hh .. 32 hh + 31, in the tile's own block
+      if (ok) {
+        const uint32_t xs = smem_u32(base + K3Smem::slot(nblk, s));
+        for (int jj = 0; jj < nblk; ++jj) {
+          const uint32_t ra = xs + (uint32_t)jj * 16384u + (uint32_t)tl * 128u;
+          // the column factor in bf16: one packed multiply per pair of channels
+          const float vref = (second && jj == ti) ? td.c2ref2 : td.c2ref;
+          const float vs = ex2(vref - td.c2[128 * jj + tl]) * td.dt[128 * jj + tl];
+          const uint32_t vv2 = pack_bf16x2(vs, vs);
+          uint32_t w[16];
+#pragma unroll
+          for (int cc = 0; cc < 4; ++cc) {
+            const uint4 in = ld_shared_v4(ra + ((uint32_t)((4 * hh + cc) ^ (tl & 7)) << 4));
+            w[4 * cc] = in.x;
+            w[4 * cc + 1] = in.y;
+            w[4 * cc + 2] = in.z;
+            w[4 * cc + 3] = in.w;
+          }
+          if (jj == ti) {
+#pragma unroll
+            for (int e = 0; e < 16; ++e) own[e] = w[e];
+          }
+          if (!steep) {
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc) {
+              uint32_t o4[4];
+#pragma unroll
+              for (int m = 0; m < 4; ++m) o4[m] = mul_bf16x2(w[4 * cc + m], vv2);
+              st_shared_v4(ra + ((uint32_t)((4 * hh + cc) ^ (tl & 7)) << 4), o4[0], o4[1], o4[2], o4[3]);
+            }
+          }
+        }
+      }
       if (k >= 2) ok = ok && mbar_wait(&ms->acc_free[a], ((k >> 1) - 1) & 1, abort_flag, err);
       // a steep head k-1 keeps its own W in this head's buffer until its MMAs are done
       if (prev_steep) ok = ok && mbar_wait(&ms->x_free[(k - 1) % NS], ((k - 1) / NS) & 1, abort_flag, err);
       prev_steep = steep;
       tc_fence_after();
       if (ok) {
-        const uint32_t xs = smem_u32(base + K3Smem::slot(nblk, s));
         const float c2t = td.c2[t];
-        // A split head's rows and sources from m = 128*ti + 64 on take the second reference,
-        // and their D x_t / u_t goes to the second intra accumulator (the first gets 0 for
-        // them, and the second gets 0 for the rows before m).
-        const bool second = td.split && tl >= 64;
         const float dsc = steep ? dh : dh * ex2((second ? td.c2ref2 : td.c2ref) - c2t);  // D / u_t
         const uint32_t acc_i = tmem + lane_off + k3_buf(a) + (second ? 128u : 64u);
-        if (td.split && ok) {  // the other intra accumulator starts from 0 in this row
+        if (td.split) {  // the other intra accumulator starts from 0 in this row
           uint32_t z[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e) z[e] = 0u;
@@ -999,46 +1033,16 @@ k_chunk_scan_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
           tmem_st16(acc_z, z);
           tmem_st16(acc_z + 16u, z);
         }
-        for (int jj = 0; jj < nblk; ++jj) {
-          const uint32_t ra = xs + (uint32_t)jj * 16384u + (uint32_t)tl * 128u;
-          // the column factor in bf16: one packed multiply per pair of channels
-          const float vref = (second && jj == ti) ? td.c2ref2 : td.c2ref;
-          const float vs = ex2(vref - td.c2[128 * jj + tl]) * td.dt[128 * jj + tl];
-          const uint32_t vv2 = pack_bf16x2(vs, vs);
-          {
-            const int half = hh;  // channels 32 half .. 32 half + 31
-            uint32_t w[16];
+        uint32_t lo[16], hi[16];
 #pragma unroll
-            for (int cc = 0; cc < 4; ++cc) {
-              const uint4 in = ld_shared_v4(ra + ((uint32_t)((4 * half + cc) ^ (tl & 7)) << 4));
-              w[4 * cc] = in.x;
-              w[4 * cc + 1] = in.y;
-              w[4 * cc + 2] = in.z;
-              w[4 * cc + 3] = in.w;
-            }
-            if (jj == ti) {
-              uint32_t lo[16], hi[16];
-#pragma unroll
-              for (int e = 0; e < 8; ++e) {
-                lo[2 * e] = __float_as_uint(__uint_as_float(w[e] << 16) * dsc);
-                lo[2 * e + 1] = __float_as_uint(__uint_as_float(w[e] & 0xffff0000u) * dsc);
-                hi[2 * e] = __float_as_uint(__uint_as_float(w[8 + e] << 16) * dsc);
-                hi[2 * e + 1] = __float_as_uint(__uint_as_float(w[8 + e] & 0xffff0000u) * dsc);
-              }
-              tmem_st16(acc_i + 32u * half, lo);
-              tmem_st16(acc_i + 32u * half + 16u, hi);
-            }
-            if (!steep) {
-#pragma unroll
-              for (int cc = 0; cc < 4; ++cc) {
-                uint32_t o4[4];
-#pragma unroll
-                for (int m = 0; m < 4; ++m) o4[m] = mul_bf16x2(w[4 * cc + m], vv2);
-                st_shared_v4(ra + ((uint32_t)((4 * half + cc) ^ (tl & 7)) << 4), o4[0], o4[1], o4[2], o4[3]);
-              }
-            }
-          }
+        for (int e = 0; e < 8; ++e) {
+          lo[2 * e] = __float_as_uint(__uint_as_float(own[e] << 16) * dsc);
+          lo[2 * e + 1] = __float_as_uint(__uint_as_float(own[e] & 0xffff0000u) * dsc);
+          hi[2 * e] = __float_as_uint(__uint_as_float(own[8 + e] << 16) * dsc);
+          hi[2 * e + 1] = __float_as_uint(__uint_as_float(own[8 + e] & 0xffff0000u) * dsc);
         }
+        tmem_st16(acc_i + 32u * hh, lo);
+        tmem_st16(acc_i + 32u * hh + 16u, hi);
         tmem_st_wait();
       }
       fence_proxy_async_smem();
