@@ -685,8 +685,9 @@ __device__ __forceinline__ TileDecay tile_decay(const float *row, int Q, int ti,
 // columns.  G (fp32, 128 * nblk columns) occupies the buffers until W_base has been built
 // from it.  A steep head builds its own W in the other head's buffer (see below).
 //
-// One thread issues a tcgen05.mma about every 110 ns whatever N is (up to 256), and several
-// issuing threads with their own accumulators run concurrently, so the products of a head
+// One thread issues a tcgen05.mma about every 67 ns at N = 64 or 128 (75-94 ns at N = 256,
+// measured), and several issuing threads with their own accumulators run concurrently
+// (three bursts of 8 complete in about the time of one), so the products of a head
 // are spread over up to three issuers of at most 8 MMAs each: C h_prev^T (warp 1), the
 // intra-chunk product of source block 0 (warp 15) and of source block 1 (warp 16).
 constexpr uint32_t K3_TM_WB = 0, K3_TM_BUF = 128, K3_BUF_COLS = 192;
