@@ -59,6 +59,8 @@ def _close(got, ref, rel):
     dict(b=1, L=37, H=4, P=16, G=2, N=32),
     dict(b=3, L=2, H=2, P=8, G=1, N=16),      # shorter than the filter
     dict(b=4, L=16390, H=2, P=32, G=1, N=16),  # long enough for the streaming kernel (ragged last range)
+    dict(b=2, L=300, H=2, P=6, G=1, N=16),     # x width a multiple of 4 channels but not of 8
+    dict(b=1, L=37, H=3, P=5, G=1, N=16),      # odd x width: one channel a thread
 ])
 def test_frontend_matches_oracle(ssd, dtype, shape):
     s = shape
