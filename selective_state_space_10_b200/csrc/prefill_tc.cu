@@ -272,22 +272,26 @@ k_chunk_state_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
         // the row, coalesced, for the chunk-scan kernel
         float4 *dst = reinterpret_cast<float4 *>(tab + (((size_t)bi * d.H + h) * nc + c) * (size_t)tab_row_floats(Q));
         for (int j = lane; j < tab_row_floats(Q) / 4; j += 32) dst[j] = reinterpret_cast<const float4 *>(row)[j];
+        __syncwarp();
+        // then, in place of dt in the shared copy, the weight the scaling below applies to
+        // each token: w_t = 2^(c2_end - c2_t) dt_t (0 past the end of the sequence)
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          if (j < per) row[kTabHdr + Q + lane * per + j] = ex2(cend - (c2v[j] + excl)) * dv[r][j];
       }
       named_barrier(1, 256);  // every head's table row is in shared memory
     }
-    // Row t of a slot is scaled by w_t = 2^(c2_end - c2_t) dt_t from its head's table row.
+    // Row t of a slot is scaled by w_t = 2^(c2_end - c2_t) dt_t, kept in its head's table row.
     for (int k = 0; k < nh; ++k) {
       const int s = k % K1_SLOTS;
       const bool ok = mbar_wait(&ms->x_full[s], (k / K1_SLOTS) & 1, abort_flag, err);
       if (ok) {
         const uint32_t xs = smem_u32(base + K1Smem::x(Q, s));
         const uint32_t ls = smem_u32(base + K1Smem::lo(Q, s));
-        const float *tr = ms->tab[k];
-        const float cend = tr[2];
-#pragma unroll 4
+        const float *tw = ms->tab[k] + kTabHdr + Q;
+#pragma unroll 8
         for (int unit = tid; unit < Q * 8; unit += 256) {
-          const int t = unit >> 3;
-          const float wv = ex2(cend - tr[kTabHdr + t]) * tr[kTabHdr + Q + t];
+          const float wv = tw[unit >> 3];
           const uint32_t off = (uint32_t)unit * 16u;  // rows are 128 B: unit*16 = row*128 + chunk*16
           const uint4 v = ld_shared_v4(xs + off);
           const uint32_t in[4] = {v.x, v.y, v.z, v.w};
