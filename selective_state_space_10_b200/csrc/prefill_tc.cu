@@ -739,16 +739,16 @@ k_chunk_scan_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
     for (int s = 0; s < K3_MAXSLOTS; ++s) {
       mbar_init(&ms->x_full[s], 1);
       mbar_init(&ms->h_full[s], 1);
-      mbar_init(&ms->ops_ready[s], 1);
+      mbar_init(&ms->ops_ready[s], 8);  // one arrival per scaling warp
       mbar_init(&ms->x_free[s], 3);  // commits of the three MMA issuers
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&ms->acc_full[a], 3);  // commits of the three MMA issuers
-      mbar_init(&ms->acc_free[a], 1);
+      mbar_init(&ms->acc_free[a], 8);  // one arrival per output warp
     }
     for (int s = 0; s < K3_CUMBUF; ++s) {
       mbar_init(&ms->tab_full[s], 1);
-      mbar_init(&ms->cum_free[s], 2);  // x/W warps + output warps
+      mbar_init(&ms->cum_free[s], 16);  // every x/W warp and every output warp
     }
     ms->abort_flag = 0;
     mbar_fence_init();
@@ -1050,10 +1050,11 @@ k_chunk_scan_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
         tmem_st16(acc_i + 32u * hh + 16u, hi);
         tmem_st_wait();
       }
+      // each warp releases its share on its own (no CTA-wide barrier in the head's loop)
       fence_proxy_async_smem();
       tc_fence_before();
-      named_barrier(1, 256);
-      if (tid == 0 && ok) {
+      __syncwarp();
+      if (lane == 0 && ok) {
         mbar_arrive(&ms->ops_ready[s]);
         mbar_arrive(&ms->cum_free[cb]);
       }
@@ -1103,8 +1104,8 @@ k_chunk_scan_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
       }
       // the accumulators and decay tables are read: release them before writing y
       tc_fence_before();
-      named_barrier(2, 256);
-      if (tid == 0 && ok) {
+      __syncwarp();
+      if (lane == 0 && ok) {
         mbar_arrive(&ms->acc_free[a]);
         mbar_arrive(&ms->cum_free[cb]);
       }
