@@ -94,46 +94,81 @@ struct K1Smem {
 };
 
 struct K1Misc {
-  uint64_t b_full, b_tmem;
+  uint64_t b_full, b_tmem[2];
   uint64_t x_full[K1_SLOTS], scaled[K1_SLOTS], x_free[K1_SLOTS];
   uint64_t acc_full[2], acc_free[2];
   uint32_t tmem;
   int abort_flag;
-  alignas(16) float tab[K1_KB_MAX][tab_row_floats(256)];  // decay table rows of the CTA's heads
+  int items_done;  // work items whose MMAs have all completed (advanced by the epilogue warps)
+  alignas(16) float tab[K1_KB_MAX][tab_row_floats(256)];  // decay table rows of the current item's heads
 };
 static_assert(offsetof(K1Misc, tab) % 16 == 0, "bulk-copy destinations must be 16-byte aligned");
 
-// TMEM columns: two accumulator slots of [high 64 | remainder 64], then B chunk^T (Q / 2).
-constexpr uint32_t K1_TM_B = 256, K1_TM_COLS = 512;  // allocation: a power of two >= 256 + Q / 2
+// TMEM columns: two accumulator slots of [high 64 | remainder 64], then two buffers for the
+// B chunk^T (Q / 2 columns each), so that the next work item's B can be moved in while the
+// current item's MMAs still read theirs.
+constexpr uint32_t K1_TM_B = 256, K1_TM_COLS = 512;  // allocation: a power of two >= 256 + Q
 
+// One work item: the heads [h0, h0 + nh) of group g for chunk c of batch row bi.
+struct K1Item {
+  int bi, c, g, h0, nh, t0, valid;
+};
+__device__ __forceinline__ K1Item k1_item(int item, const Dims &d, int Q, int nc, int kb, int nhb) {
+  K1Item w;
+  const int hb = item % nhb;
+  item /= nhb;
+  w.g = item % d.G;
+  item /= d.G;
+  w.c = item % nc;
+  w.bi = item / nc;
+  w.h0 = w.g * d.hpg + hb * kb;
+  w.nh = min(kb, d.hpg - hb * kb);
+  w.t0 = w.c * Q;
+  w.valid = min(Q, d.L - w.t0);
+  return w;
+}
+
+// Bounded wait for a counter in shared memory to reach `target` (sleeping between checks);
+// gives up like mbar_wait.
+__device__ __forceinline__ bool k1_wait_count(volatile int *cnt, int target, volatile int *abort, int *err) {
+  if (*cnt >= target) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (*cnt < target) {
+    if (*abort) return false;
+    if (globaltimer_ns() - t0 > 2000000000ull) {
+      *abort = 1;
+      if (err) atomicExch(err, 1);
+      return false;
+    }
+    __nanosleep(128);
+  }
+  return true;
+}
+
+// kPersist: a persistent grid for launches with more work items than SMs: CTA j takes items
+// j, j + gridDim.x, ... in turn, each role carrying its ring and accumulator counters from
+// one item to the next, so that the next item's B chunk, decay tables and first x tiles
+// load while the current item's last heads are still being multiplied and written out.
+// Otherwise one item per CTA (a compile-time single pass of the same code).
+template <bool kPersist>
 __global__ void __launch_bounds__(K1_THREADS, 1)
 k_chunk_state_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_B,
                  const float *__restrict__ dt, const float *__restrict__ A, const float *__restrict__ D,
                  float *__restrict__ tab, float *__restrict__ cdecay, float *__restrict__ states, int *err, Dims d, int Q,
-                 int nc, int kb, int nhb) {
+                 int nc, int kb, int nhb, int nitems) {
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte aligned, and derived from the shared array itself (no integer round trip),
   // so that the compiler keeps every access through it in the shared address space
   uint8_t *base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   K1Misc *ms = reinterpret_cast<K1Misc *>(base + K1Smem::misc(Q));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-
-  // work item: (bi, c, g, hb) with hb fastest
-  int item = blockIdx.x;
-  const int hb = item % nhb;
-  item /= nhb;
-  const int g = item % d.G;
-  item /= d.G;
-  const int c = item % nc;
-  const int bi = item / nc;
-  const int h0 = g * d.hpg + hb * kb;
-  const int nh = min(kb, d.hpg - hb * kb);
-  const int t0 = c * Q;
-  const int valid = min(Q, d.L - t0);
+  const int my_items = kPersist ? ((int)blockIdx.x < nitems ? (nitems - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0) : 1;
+  auto item_of = [&](int i) { return k1_item((int)blockIdx.x + i * (int)gridDim.x, d, Q, nc, kb, nhb); };
 
   if (threadIdx.x == 0) {
     mbar_init(&ms->b_full, 1);
-    mbar_init(&ms->b_tmem, 1);
+    mbar_init(&ms->b_tmem[0], 1);
+    mbar_init(&ms->b_tmem[1], 1);
     for (int s = 0; s < K1_SLOTS; ++s) {
       mbar_init(&ms->x_full[s], 1);
       mbar_init(&ms->scaled[s], 1);
@@ -144,6 +179,7 @@ k_chunk_state_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
       mbar_init(&ms->acc_free[a], 1);
     }
     ms->abort_flag = 0;
+    ms->items_done = 0;
     mbar_fence_init();
   }
   if (warp == 1) {
@@ -169,24 +205,43 @@ k_chunk_state_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
 
   if (warp == 0) {
     // ------------------------------------------------------------- TMA producer
+    // Slot K1_SLOTS - 1 also takes each item's B chunk: after the slot's last x has been
+    // consumed and the previous B has been moved to TMEM; its next x waits for this B's move.
     if (lane == 0) {
       tma_prefetch_desc(&tm_x);
       tma_prefetch_desc(&tm_B);
-      mbar_arrive_expect_tx(&ms->b_full, 2u * Q * 128u);
-      tma_load_3d(base + K1Smem::bm(Q), &tm_B, &ms->b_full, g * TN, t0, bi);
-      tma_load_3d(base + K1Smem::bm(Q) + (uint32_t)Q * 128u, &tm_B, &ms->b_full, g * TN + 64, t0, bi);
-      int issued = 0;
-      for (int k = 0; k < nh; ++k) {
-        const int s = k % K1_SLOTS, u = k / K1_SLOTS;
-        if (k >= K1_SLOTS && !mbar_wait(&ms->x_free[s], (u - 1) & 1, abort_flag, err)) break;
-        // the last slot holds the B chunk until it has been moved to TMEM
-        if (k == K1_SLOTS - 1 && !mbar_wait(&ms->b_tmem, 0, abort_flag, err)) break;
-        mbar_arrive_expect_tx(&ms->x_full[s], (uint32_t)Q * 128u);
-        tma_load_3d(base + K1Smem::x(Q, s), &tm_x, &ms->x_full[s], (h0 + k) * TP, t0, bi);
-        issued = k + 1;
+      int gk = 0, issued = 0, nb = 0, last = -1;  // last: global head index of slot K1_SLOTS-1's last x
+      bool ok = true;
+      for (int i = 0; ok && i < my_items; ++i) {
+        const K1Item w = item_of(i);
+        if (i > 0 && !mbar_wait(&ms->b_tmem[(i - 1) & 1], ((i - 1) >> 1) & 1, abort_flag, err)) break;
+        if (last >= 0 && !mbar_wait(&ms->x_free[K1_SLOTS - 1], (last / K1_SLOTS) & 1, abort_flag, err)) break;
+        mbar_arrive_expect_tx(&ms->b_full, 2u * Q * 128u);
+        tma_load_3d(base + K1Smem::bm(Q), &tm_B, &ms->b_full, w.g * TN, w.t0, w.bi);
+        tma_load_3d(base + K1Smem::bm(Q) + (uint32_t)Q * 128u, &tm_B, &ms->b_full, w.g * TN + 64, w.t0, w.bi);
+        nb = i + 1;
+        bool b_in_slot = true;
+        for (int k = 0; k < w.nh; ++k, ++gk) {
+          const int s = gk % K1_SLOTS, u = gk / K1_SLOTS;
+          if (gk >= K1_SLOTS && !mbar_wait(&ms->x_free[s], (u - 1) & 1, abort_flag, err)) {
+            ok = false;
+            break;
+          }
+          if (s == K1_SLOTS - 1 && b_in_slot) {
+            if (!mbar_wait(&ms->b_tmem[i & 1], (i >> 1) & 1, abort_flag, err)) {
+              ok = false;
+              break;
+            }
+            b_in_slot = false;
+          }
+          mbar_arrive_expect_tx(&ms->x_full[s], (uint32_t)Q * 128u);
+          tma_load_3d(base + K1Smem::x(Q, s), &tm_x, &ms->x_full[s], (w.h0 + k) * TP, w.t0, w.bi);
+          if (s == K1_SLOTS - 1) last = gk;
+          issued = gk + 1;
+        }
       }
       if (*abort_flag) {  // let this CTA's own loads land before it exits
-        mbar_wait_drain(&ms->b_full, 0);
+        if (nb > 0) mbar_wait_drain(&ms->b_full, (uint32_t)((nb - 1) & 1));
         for (int k = (issued > K1_SLOTS ? issued - K1_SLOTS : 0); k < issued; ++k)
           mbar_wait_drain(&ms->x_full[k % K1_SLOTS], (k / K1_SLOTS) & 1);
       }
@@ -197,132 +252,178 @@ k_chunk_state_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
     if (lane == 0) {
       // A = B chunk^T from TMEM: [M = d_state lanes][K = token], bf16 pairs along K
       const uint32_t idesc = idesc_bf16_f32(128, 2 * TP, /*a MN-major*/ false, /*b MN-major*/ true);
-      bool ok = mbar_wait(&ms->b_tmem, 0, abort_flag, err);
-      for (int k = 0; ok && k < nh; ++k) {
-        const int s = k % K1_SLOTS, a = k & 1;
-        if (!mbar_wait(&ms->scaled[s], (k / K1_SLOTS) & 1, abort_flag, err)) break;
-        if (k >= 2 && !mbar_wait(&ms->acc_free[a], ((k >> 1) - 1) & 1, abort_flag, err)) break;
-        tc_fence_after();
-        const uint32_t x_addr = smem_u32(base + K1Smem::x(Q, s));
-        for (int ks = 0; ks < Q / 16; ++ks) {
-          // B = [K = token][N = (high | remainder) x channel]: two 64-wide blocks Q*128 B apart
-          const uint64_t bd = smem_desc_sw128(x_addr + ks * 2048u, (uint32_t)Q * 128u, 1024u);
-          mma_bf16_ts(tmem + (uint32_t)(a * 2 * TP), tmem + K1_TM_B + 8u * ks, bd, idesc, ks > 0 ? 1u : 0u);
+      int gk = 0;
+      bool ok = true;
+      for (int i = 0; ok && i < my_items; ++i) {
+        const K1Item w = item_of(i);
+        if (!(ok = mbar_wait(&ms->b_tmem[i & 1], (i >> 1) & 1, abort_flag, err))) break;
+        const uint32_t bcol = K1_TM_B + (uint32_t)(i & 1) * (uint32_t)(Q / 2);
+        for (int k = 0; k < w.nh; ++k, ++gk) {
+          const int s = gk % K1_SLOTS, a = gk & 1;
+          if (!(ok = mbar_wait(&ms->scaled[s], (gk / K1_SLOTS) & 1, abort_flag, err))) break;
+          if (gk >= 2 && !(ok = mbar_wait(&ms->acc_free[a], ((gk >> 1) - 1) & 1, abort_flag, err))) break;
+          tc_fence_after();
+          const uint32_t x_addr = smem_u32(base + K1Smem::x(Q, s));
+          for (int ks = 0; ks < Q / 16; ++ks) {
+            // B = [K = token][N = (high | remainder) x channel]: two 64-wide blocks Q*128 B apart
+            const uint64_t bd = smem_desc_sw128(x_addr + ks * 2048u, (uint32_t)Q * 128u, 1024u);
+            mma_bf16_ts(tmem + (uint32_t)(a * 2 * TP), tmem + bcol + 8u * ks, bd, idesc, ks > 0 ? 1u : 0u);
+          }
+          mma_commit(&ms->acc_full[a]);
+          mma_commit(&ms->x_free[s]);
         }
-        mma_commit(&ms->acc_full[a]);
-        mma_commit(&ms->x_free[s]);
       }
     }
     __syncwarp();
   } else if (warp < 10) {
     // ------------------------------------------------------------- scale warps (256 threads)
     const int tid = threadIdx.x - 64, wl = warp - 2;
-    {
-      // Decay tables first (per-chunk dt.A cumulative sums), one head per warp and round:
-      // every lane sums Q/32 consecutive tokens, a shuffle scan adds the lanes' totals.
-      // All loads of both rounds are issued before the first use.
-      const int per = Q / 32;
-      float dv[2][8], av[2] = {0.f, 0.f}, dd[2] = {0.f, 0.f};
+    int gk = 0;
+    bool ok = true;
+    for (int i = 0; i < my_items; ++i) {
+      const K1Item w = item_of(i);
+      const int bi = w.bi, c = w.c, h0 = w.h0, nh = w.nh, t0 = w.t0, valid = w.valid;
+      {
+        // Decay tables first (per-chunk dt.A cumulative sums), one head per warp and round:
+        // every lane sums Q/32 consecutive tokens, a shuffle scan adds the lanes' totals.
+        // All loads of both rounds are issued before the first use.  The previous item's
+        // rows are no longer read: these warps have scaled all of its heads.
+        const int per = Q / 32;
+        float dv[2][8], av[2] = {0.f, 0.f}, dd[2] = {0.f, 0.f};
 #pragma unroll
-      for (int r = 0; r < 2; ++r) {
-        const int k = wl + 8 * r, h = h0 + k;
+        for (int r = 0; r < 2; ++r) {
+          const int k = wl + 8 * r, h = h0 + k;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const int t = lane * per + j;
-          dv[r][j] = (k < nh && j < per && t < valid) ? __ldg(dt + ((size_t)bi * d.L + t0 + t) * d.H + h) : 0.f;
-        }
-        if (k < nh) {
-          av[r] = __ldg(A + h);
-          dd[r] = __ldg(D + h);
-        }
-      }
-#pragma unroll
-      for (int r = 0; r < 2; ++r) {
-        const int k = wl + 8 * r, h = h0 + k;
-        if (k >= nh) break;
-        const float a2 = av[r] * kLog2e;
-        float c2v[8];
-        float run = 0.f;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          run += dv[r][j] * a2;
-          c2v[j] = run;
-        }
-        float incl = run;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const float u = __shfl_up_sync(0xffffffffu, incl, o);
-          if (lane >= o) incl += u;
-        }
-        const float excl = incl - run;
-        const float cend = __shfl_sync(0xffffffffu, incl, 31);
-        float *row = ms->tab[k];
-#pragma unroll
-        for (int j = 0; j < 8; ++j)
-          if (j < per) {
-            row[kTabHdr + lane * per + j] = c2v[j] + excl;
-            row[kTabHdr + Q + lane * per + j] = dv[r][j];
+          for (int j = 0; j < 8; ++j) {
+            const int t = lane * per + j;
+            dv[r][j] = (k < nh && j < per && t < valid) ? __ldg(dt + ((size_t)bi * d.L + t0 + t) * d.H + h) : 0.f;
           }
-        if (lane == 0) {
-          const float dec = ex2(cend);
-          *reinterpret_cast<float4 *>(row) = make_float4(dd[r], dec, cend, 0.f);
-          cdecay[((size_t)bi * d.H + h) * nc + c] = dec;
+          if (k < nh) {
+            av[r] = __ldg(A + h);
+            dd[r] = __ldg(D + h);
+          }
         }
-        __syncwarp();
-        // the row, coalesced, for the chunk-scan kernel
-        float4 *dst = reinterpret_cast<float4 *>(tab + (((size_t)bi * d.H + h) * nc + c) * (size_t)tab_row_floats(Q));
-        for (int j = lane; j < tab_row_floats(Q) / 4; j += 32) dst[j] = reinterpret_cast<const float4 *>(row)[j];
-        __syncwarp();
-        // then, in place of dt in the shared copy, the weight the scaling below applies to
-        // each token: w_t = 2^(c2_end - c2_t) dt_t (0 past the end of the sequence)
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
-          if (j < per) row[kTabHdr + Q + lane * per + j] = ex2(cend - (c2v[j] + excl)) * dv[r][j];
+        for (int r = 0; r < 2; ++r) {
+          const int k = wl + 8 * r, h = h0 + k;
+          if (k >= nh) break;
+          const float a2 = av[r] * kLog2e;
+          float c2v[8];
+          float run = 0.f;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            run += dv[r][j] * a2;
+            c2v[j] = run;
+          }
+          float incl = run;
+#pragma unroll
+          for (int o = 1; o < 32; o <<= 1) {
+            const float uu = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += uu;
+          }
+          const float excl = incl - run;
+          const float cend = __shfl_sync(0xffffffffu, incl, 31);
+          float *row = ms->tab[k];
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            if (j < per) {
+              row[kTabHdr + lane * per + j] = c2v[j] + excl;
+              row[kTabHdr + Q + lane * per + j] = dv[r][j];
+            }
+          if (lane == 0) {
+            const float dec = ex2(cend);
+            *reinterpret_cast<float4 *>(row) = make_float4(dd[r], dec, cend, 0.f);
+            cdecay[((size_t)bi * d.H + h) * nc + c] = dec;
+          }
+          __syncwarp();
+          // the row, coalesced, for the chunk-scan kernel
+          float4 *dst = reinterpret_cast<float4 *>(tab + (((size_t)bi * d.H + h) * nc + c) * (size_t)tab_row_floats(Q));
+          for (int j = lane; j < tab_row_floats(Q) / 4; j += 32) dst[j] = reinterpret_cast<const float4 *>(row)[j];
+          __syncwarp();
+          // then, in place of dt in the shared copy, the weight the scaling below applies to
+          // each token: w_t = 2^(c2_end - c2_t) dt_t (0 past the end of the sequence)
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            if (j < per) row[kTabHdr + Q + lane * per + j] = ex2(cend - (c2v[j] + excl)) * dv[r][j];
+        }
       }
-      named_barrier(1, 256);  // every head's table row is in shared memory
-    }
-    // Row t of a slot is scaled by w_t = 2^(c2_end - c2_t) dt_t, kept in its head's table row.
-    for (int k = 0; k < nh; ++k) {
-      const int s = k % K1_SLOTS;
-      const bool ok = mbar_wait(&ms->x_full[s], (k / K1_SLOTS) & 1, abort_flag, err);
-      if (ok) {
-        const uint32_t xs = smem_u32(base + K1Smem::x(Q, s));
-        const uint32_t ls = smem_u32(base + K1Smem::lo(Q, s));
-        const float *tw = ms->tab[k] + kTabHdr + Q;
+      // The B chunk into its TMEM buffer (i & 1) as the MMA's A operand, once it has landed
+      // and once the item that last used the buffer (i - 2) has finished its MMAs: lane n
+      // gets B[t][n] for every token, packed in pairs (t even in the low half), the two
+      // warps of a TMEM lane quarter taking half of the columns each.  In shared memory
+      // (128-byte swizzle) 16-byte chunk j of row t of a 64-wide block sits at chunk j ^ (t & 7).
+      // (The first item's B is moved by the epilogue warps, idle until its first head, so
+      // that the move overlaps these tables.)
+      if (i > 0) ok = ok && mbar_wait(&ms->b_full, (uint32_t)(i & 1), abort_flag, err);
+      ok = ok && (i < 2 || k1_wait_count(&ms->items_done, i - 1, abort_flag, err));
+      tc_fence_after();
+      if (ok && i > 0) {
+        const int q = warp & 3, half = wl >> 2;
+        const int n = q * 32 + lane;
+        const uint32_t src = smem_u32(base + K1Smem::bm(Q)) + (uint32_t)(n >> 6) * (uint32_t)Q * 128u +
+                             (uint32_t)(n & 7) * 2u;
+        const uint32_t j8 = (uint32_t)((n & 63) >> 3);
+        const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+        const uint32_t bcol = K1_TM_B + (uint32_t)(i & 1) * (uint32_t)(Q / 2);
+        for (int c0 = half * (Q / 4); c0 < (half + 1) * (Q / 4); c0 += 16) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const uint32_t t = 2u * (uint32_t)(c0 + e);
+            const uint32_t b0 = ld_shared_u16(src + t * 128u + ((j8 ^ (t & 7u)) << 4));
+            const uint32_t b1 = ld_shared_u16(src + (t + 1u) * 128u + ((j8 ^ ((t + 1u) & 7u)) << 4));
+            pk[e] = b0 | (b1 << 16);
+          }
+          tmem_st16(tmem + lane_off + bcol + (uint32_t)c0, pk);
+        }
+        tmem_st_wait();
+      }
+      fence_proxy_async_smem();  // the slot is refilled by TMA after these reads
+      tc_fence_before();
+      named_barrier(1, 256);  // every head's table row is in shared memory, B is in TMEM
+      if (tid == 0 && ok && i > 0) mbar_arrive(&ms->b_tmem[i & 1]);
+      // Row t of a slot is scaled by w_t = 2^(c2_end - c2_t) dt_t, kept in its head's table row.
+      for (int k = 0; k < nh; ++k, ++gk) {
+        const int s = gk % K1_SLOTS;
+        ok = ok && mbar_wait(&ms->x_full[s], (gk / K1_SLOTS) & 1, abort_flag, err);
+        if (ok) {
+          const uint32_t xs = smem_u32(base + K1Smem::x(Q, s));
+          const uint32_t ls = smem_u32(base + K1Smem::lo(Q, s));
+          const float *tw = ms->tab[k] + kTabHdr + Q;
 #pragma unroll 8
-        for (int unit = tid; unit < Q * 8; unit += 256) {
-          const float wv = tw[unit >> 3];
-          const uint32_t off = (uint32_t)unit * 16u;  // rows are 128 B: unit*16 = row*128 + chunk*16
-          const uint4 v = ld_shared_v4(xs + off);
-          const uint32_t in[4] = {v.x, v.y, v.z, v.w};
-          uint32_t hi[4], rem[4];
+          for (int unit = tid; unit < Q * 8; unit += 256) {
+            const float wv = tw[unit >> 3];
+            const uint32_t off = (uint32_t)unit * 16u;  // rows are 128 B: unit*16 = row*128 + chunk*16
+            const uint4 v = ld_shared_v4(xs + off);
+            const uint32_t in[4] = {v.x, v.y, v.z, v.w};
+            uint32_t hi[4], rem[4];
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const float a0 = __uint_as_float(in[q] << 16) * wv;  // exact x * w in fp32
-            const float a1 = __uint_as_float(in[q] & 0xffff0000u) * wv;
-            // high part: the top 16 bits (truncation), so a - high is exact in fp32 and is
-            // rounded once, to the bf16 remainder
-            const uint32_t b0 = __float_as_uint(a0) & 0xffff0000u, b1 = __float_as_uint(a1) & 0xffff0000u;
-            hi[q] = __byte_perm(b0, b1, 0x7632);
-            rem[q] = pack_bf16x2(a0 - __uint_as_float(b0), a1 - __uint_as_float(b1));
+            for (int qq = 0; qq < 4; ++qq) {
+              const float a0 = __uint_as_float(in[qq] << 16) * wv;  // exact x * w in fp32
+              const float a1 = __uint_as_float(in[qq] & 0xffff0000u) * wv;
+              // high part: the top 16 bits (truncation), so a - high is exact in fp32 and is
+              // rounded once, to the bf16 remainder
+              const uint32_t b0 = __float_as_uint(a0) & 0xffff0000u, b1 = __float_as_uint(a1) & 0xffff0000u;
+              hi[qq] = __byte_perm(b0, b1, 0x7632);
+              rem[qq] = pack_bf16x2(a0 - __uint_as_float(b0), a1 - __uint_as_float(b1));
+            }
+            st_shared_v4(xs + off, hi[0], hi[1], hi[2], hi[3]);
+            st_shared_v4(ls + off, rem[0], rem[1], rem[2], rem[3]);
           }
-          st_shared_v4(xs + off, hi[0], hi[1], hi[2], hi[3]);
-          st_shared_v4(ls + off, rem[0], rem[1], rem[2], rem[3]);
         }
+        fence_proxy_async_smem();
+        named_barrier(1, 256);
+        if (tid == 0 && ok) mbar_arrive(&ms->scaled[s]);
       }
-      fence_proxy_async_smem();
-      named_barrier(1, 256);
-      if (tid == 0 && ok) mbar_arrive(&ms->scaled[s]);
     }
   } else {
     // ------------------------------------------------------------- epilogue warps (128 threads)
     const int q = warp & 3;
     const int n = q * 32 + lane;  // d_state row of the accumulator
     const int tid = threadIdx.x - 320;
-    {
-      // First move the B chunk into TMEM as the MMA's A operand: lane n gets B[t][n] for
-      // every token, packed in pairs (t even in the low half).  In shared memory (128-byte
-      // swizzle) 16-byte chunk j of row t of a 64-wide block sits at chunk j ^ (t & 7).
+    if (my_items > 0) {
+      // The first item's B chunk into TMEM buffer 0 (later items' are moved by the scale
+      // warps): lane n gets B[t][n] for every token, packed in pairs.
       bool ok = mbar_wait(&ms->b_full, 0, abort_flag, err);
       if (ok) {
         const uint32_t src = smem_u32(base + K1Smem::bm(Q)) + (uint32_t)(n >> 6) * (uint32_t)Q * 128u +
@@ -345,28 +446,34 @@ k_chunk_state_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
       fence_proxy_async_smem();  // the slot is refilled by TMA after these reads
       tc_fence_before();
       named_barrier(2, 128);
-      if (tid == 0 && ok) mbar_arrive(&ms->b_tmem);
+      if (tid == 0 && ok) mbar_arrive(&ms->b_tmem[0]);
     }
-    for (int k = 0; k < nh; ++k) {
-      const int a = k & 1, h = h0 + k;
-      const bool ok = mbar_wait(&ms->acc_full[a], (k >> 1) & 1, abort_flag, err);
-      tc_fence_after();
-      if (ok) {
-        // S in the layout of the entering states: [n / 64][p][n % 64] per (batch, chunk, head)
-        float *out = states + (((size_t)bi * nc + c) * d.H + h) * (size_t)(TP * TN) + (n >> 6) * (TP * 64) + (n & 63);
+    int gk = 0;
+    for (int i = 0; i < my_items; ++i) {
+      const K1Item w = item_of(i);
+      for (int k = 0; k < w.nh; ++k, ++gk) {
+        const int a = gk & 1, h = w.h0 + k;
+        const bool ok = mbar_wait(&ms->acc_full[a], (gk >> 1) & 1, abort_flag, err);
+        tc_fence_after();
+        if (ok) {
+          // S in the layout of the entering states: [n / 64][p][n % 64] per (batch, chunk, head)
+          float *out = states + (((size_t)w.bi * nc + w.c) * d.H + h) * (size_t)(TP * TN) + (n >> 6) * (TP * 64) + (n & 63);
 #pragma unroll
-        for (int cg = 0; cg < 2; ++cg) {
-          float vh[32], vl[32];
-          tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(a * 2 * TP + cg * 32), vh);
-          tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(a * 2 * TP + TP + cg * 32), vl);
-          tmem_ld_wait();
+          for (int cg = 0; cg < 2; ++cg) {
+            float vh[32], vl[32];
+            tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(a * 2 * TP + cg * 32), vh);
+            tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(a * 2 * TP + TP + cg * 32), vl);
+            tmem_ld_wait();
 #pragma unroll
-          for (int j = 0; j < 32; ++j) out[(size_t)(cg * 32 + j) * 64] = vh[j] + vl[j];
+            for (int j = 0; j < 32; ++j) out[(size_t)(cg * 32 + j) * 64] = vh[j] + vl[j];
+          }
         }
+        tc_fence_before();
+        named_barrier(2, 128);
+        if (tid == 0) mbar_arrive(&ms->acc_free[a]);
       }
-      tc_fence_before();
-      named_barrier(2, 128);
-      if (tid == 0) mbar_arrive(&ms->acc_free[a]);
+      // every MMA of item i has completed (each head's completion was seen above)
+      if (tid == 0) *reinterpret_cast<volatile int *>(&ms->items_done) = i + 1;
     }
   }
 
@@ -1068,7 +1175,6 @@ k_chunk_scan_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant_
     const int q = warp & 3, hf = (warp - 6) >> 2;
     const int tl = q * 32 + lane;
     const int t = 128 * ti + tl;
-    const int tid = threadIdx.x - 192;
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
     uint8_t *stg = base + K3Smem::ystage(warp - 6);
     const uint32_t srow = smem_u32(stg) + (uint32_t)lane * 128u;
@@ -1291,7 +1397,9 @@ cudaError_t set_smem_limits_once() {
   if (e != cudaSuccess) return e;
   const uint64_t bit = dev < 64 ? (uint64_t)1 << dev : 0;
   if (bit && (done.load(std::memory_order_acquire) & bit)) return cudaSuccess;
-  e = cudaFuncSetAttribute(k_chunk_state_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)k1_smem_bytes(256));
+  e = cudaFuncSetAttribute(k_chunk_state_tc<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)k1_smem_bytes(256));
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(k_chunk_state_tc<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)k1_smem_bytes(256));
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(k_chunk_scan_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kK3SmemBytes);
   if (e == cudaSuccess)
@@ -1442,8 +1550,13 @@ cudaError_t launch_tc_prefill(const __nv_bfloat16 *x, const float *dt, const flo
     const int base_items = d.b * nc * d.G;
     const int kb = std::min(K1_KB_MAX, pick_heads_per_cta(base_items, d.hpg, sms, 1.0));
     const int nhb = (d.hpg + kb - 1) / kb;
-    e = launch_after(dim3((unsigned)(base_items * nhb)), K1_THREADS, tc_prefill_smem_k1(Q), st, pdl, k_chunk_state_tc,
-                     tm_x1, tm_B1, dt, A, D, tab, cdecay, states, err, d, Q, nc, kb, nhb);
+    const int nitems = base_items * nhb;
+    if (nitems > sms)  // more items than SMs: a persistent grid, one CTA per SM
+      e = launch_after(dim3((unsigned)sms), K1_THREADS, tc_prefill_smem_k1(Q), st, pdl, k_chunk_state_tc<true>, tm_x1,
+                       tm_B1, dt, A, D, tab, cdecay, states, err, d, Q, nc, kb, nhb, nitems);
+    else
+      e = launch_after(dim3((unsigned)nitems), K1_THREADS, tc_prefill_smem_k1(Q), st, pdl, k_chunk_state_tc<false>,
+                       tm_x1, tm_B1, dt, A, D, tab, cdecay, states, err, d, Q, nc, kb, nhb, nitems);
     if (e != cudaSuccess) return e;
   }
   if ((e = mark(1)) != cudaSuccess) return e;

@@ -75,6 +75,19 @@ def test_prefill_shapes(ssd, dtype, shape):
     check_prefill(ssd, si, s["Q"], f"{dtype} {s}")
 
 
+@pytest.mark.parametrize("shape", [
+    dict(b=2, L=128 * 100 + 5, H=4, G=2, Q=128),   # 404 work items of one head pair, ragged last chunk
+    dict(b=1, L=256 * 30 + 200, H=26, G=1, Q=256),  # 279 items of 3 heads (the last block 2), ragged last chunk
+])
+def test_prefill_more_work_items_than_sms(ssd, shape):
+    """Tensor-core prefills whose chunk-state launch has more work items than the GPU has
+    SMs (the persistent grid, each CTA taking several items in turn), checked in full
+    against the oracle."""
+    s = shape
+    si = inputs.sequence(s["b"], s["L"], s["H"], 64, 128, s["G"], "bf16", seed=321)
+    check_prefill(ssd, si, s["Q"], f"bf16 {s}")
+
+
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
 @pytest.mark.parametrize("chunk", [1, 2, 16, 32, 64, 128, 256])
 def test_chunk_sizes(ssd, dtype, chunk):
