@@ -399,8 +399,10 @@ def prefill_leg(args, dev, rank, world, peaks, sampler):
     sampler.active(True)
     ha, hb = mk(), mk()
     ha.record(stream)
+    tq = time.perf_counter()
     for k in range(K):
         calls[k % nsets]()
+    host_us = (time.perf_counter() - tq) / K * 1e6  # enqueue time per call (the GPU runs behind)
     hb.record(stream)
     torch.cuda.synchronize(dev)
     barrier(world, dev)
@@ -483,6 +485,7 @@ def prefill_leg(args, dev, rank, world, peaks, sampler):
                 "frac": min_bytes / secs / 1e9 / peaks["hbm_gbs"], "peak": peaks["hbm_gbs"]},
         "serial_ms_per_step": serial_ms,
         "rotated_copies_outputs_identical": bool(rotated_same),
+        "host_enqueue_us_per_call": host_us,
         "single_step_l2_flushed": {"ms_per_step": statistics.mean(step_ms),
                                    "what": "one prefill after a 256 MiB write that evicts L2, an event on each side"},
         "kernels": {n: {"avg_ms": avg[n], "share": avg[n] / tot,
@@ -944,6 +947,7 @@ def run_ours(args):
         "gpu_launches_prefill_timed_region": pre["gpu_launches"], "e2e": pre["e2e"],
         "single_step_l2_flushed": pre["single_step_l2_flushed"],
         "rotated_copies_outputs_identical": pre["rotated_copies_outputs_identical"],
+        "host_enqueue_us_per_call": pre["host_enqueue_us_per_call"],
         "l2_clean_context": pre["l2_clean_context"], "peaks": peaks, "clocks": sampler.summary(), "impl": "ours",
     }
     if dec:
